@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Benchmark of the fused SVDQuant W4A4 linear (quantizer + block-scaled FP4 GEMM
+with the rank-R epilogue) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = one full forward of the layer (both kernels) on one batch of the
+workload (default: the diffusion-transformer attention projection, M=4096,
+K=N=3072, R=32, synthetic seeded inputs).  Prints one JSON line.
+
+Timing: 8 replica sets (own weights, x, y, workspace) rotate so that the
+working set (~0.5 GB) is far larger than the 126 MB L2 and every step reads
+its inputs from HBM.  The K timed steps are one CUDA-graph replay bracketed by
+CUDA events on the launching stream (barrier + synchronize on both sides);
+per-kernel averages come from graphs of each stage alone over the same sets.
+Multi-GPU (torchrun): independent replicas, one per rank, no collective on the
+data path ("replicas only"); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor throughput ratio on B200 (9 / 2.25 PFLOP/s)
+N_SETS = 8
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def flops_per_step(M, K, N, R):
+    return 2.0 * M * N * K + 2.0 * M * K * R + 2.0 * M * N * R
+
+
+def quant_bytes(M, K, R):
+    # x read, codes + scales + L written, proj_down + smooth read (algorithmic).
+    return 2.0 * M * K + M * K / 2 + M * K / 16 + 2.0 * M * R + 2.0 * K * R + 2.0 * K
+
+
+def gemm_bytes(M, K, N, R):
+    # codes + scales + L read, weights (codes + scales + proj_up + alpha) read, y written.
+    return M * K / 2 + M * K / 16 + 2.0 * M * R + N * K / 2 + N * K / 16 + 2.0 * N * R + 4.0 * N + 2.0 * M * N
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = None
+            try:
+                uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            except Exception:
+                pass
+            h = None
+            if uuid:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+                except Exception:
+                    h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._nvml, self._h = pynvml, h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+
+    def _run(self):
+        n = self._nvml
+        names = {
+            "hw_slowdown": getattr(n, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "hw_thermal_slowdown": getattr(n, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "sw_thermal_slowdown": getattr(n, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "sw_power_cap": getattr(n, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_power_brake_slowdown": getattr(n, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+                r = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for k, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "source": "nvml, 2 ms period, during the timed region"}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, value):
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_oracle_run(ck, rows):
+    from oracle import svdq_oracle as O
+    t0 = time.perf_counter()
+    y = O.linear_forward(ck, rows=rows)
+    dt = time.perf_counter() - t0
+    return y, dt
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def run_reference(args, world, rank):
+    """The oracle as it stands, timed on the host cores (bounded row sample per step)."""
+    from bit_quantized_linear_svdq_b200 import synthetic
+    if rank != 0:
+        return
+    ck = synthetic.load(args.workload)
+    rows = np.arange(min(ck.M, args.ref_rows))
+    cpu_oracle_run(ck, rows[: min(16, len(rows))])          # warm caches / BLAS threads
+    times = []
+    for _ in range(max(1, args.warmup if args.warmup < 3 else 1)):
+        cpu_oracle_run(ck, rows)
+    for _ in range(args.steps):
+        _, dt = cpu_oracle_run(ck, rows)
+        times.append(dt)
+    t = sum(times) / len(times)
+    fl = flops_per_step(len(rows), ck.K, ck.N, ck.R)
+    value = fl / t / 1e12
+    cores = cpu_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(ck, extra={"sample_rows": len(rows)}),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{len(rows)} of {ck.M} token rows of the workload per step "
+                                   f"(numpy fp64 GEMM over dequantized NVFP4 + fp32-emulated quantizer)"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+METRIC = "W4A4+low-rank linear TFLOPS & % of dense-FP4 roofline at M=4096,K=N=3072,R=32"
+
+
+def config_of(ck, extra=None):
+    c = {"workload": ck.name, "M": ck.M, "K": ck.K, "N": ck.N, "R": ck.R, "rotate_block": ck.rotate_block,
+         "l2": f"inputs rotate over {N_SETS} replica sets (~{N_SETS} x working set) > 126 MB L2",
+         "parallelism": "replicas"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def run_ours(args, world, rank, local):
+    import bit_quantized_linear_svdq_b200 as S
+    from bit_quantized_linear_svdq_b200 import synthetic
+
+    S.load_library()
+    ck = synthetic.load(args.workload)
+    M, K, N, R = ck.M, ck.K, ck.N, ck.R
+    if ck.qweight is None:
+        raise SystemExit("bench workloads must carry a quantized checkpoint")
+
+    def dev(bits, dtype):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16 if dtype == torch.bfloat16 else np.uint8)) \
+            .view(dtype).cuda()
+
+    sets = []
+    for i in range(N_SETS):
+        layer = S.SVDQLinear(dev(ck.qweight, torch.uint8), dev(ck.wscales, torch.uint8),
+                             dev(ck.proj_down, torch.bfloat16), dev(ck.proj_up, torch.bfloat16),
+                             dev(ck.smooth_factor, torch.bfloat16), dev(ck.wcscales, torch.bfloat16),
+                             dev(ck.wtscale, torch.bfloat16), rotate_block=ck.rotate_block)
+        x = dev(ck.x, torch.bfloat16)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(S.svdq_workspace_bytes(layer.handle, M), dtype=torch.uint8, device="cuda")
+        sets.append((layer, x, y, ws))
+    stream = torch.cuda.Stream()
+
+    def step(i, which="both"):
+        layer, x, y, ws = sets[i % N_SETS]
+        if which in ("both", "quant"):
+            S.svdq_linear_forward_quantize(layer.handle, x.data_ptr(), M, ws.data_ptr(), stream)
+        if which in ("both", "gemm"):
+            S.svdq_linear_forward_gemm(layer.handle, M, y.data_ptr(), ws.data_ptr(), stream)
+
+    def graph_of(n, which):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            for i in range(N_SETS):                 # eager pass: attributes set, sets initialised
+                step(i, which)
+            stream.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n):
+                    step(i, which)
+        return g
+
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            step(i)
+    torch.cuda.synchronize()
+    g_full = graph_of(args.steps, "both")
+    g_quant = graph_of(args.steps, "quant")
+    g_gemm = graph_of(args.steps, "gemm")
+    for g in (g_full, g_quant, g_gemm):        # graph warm-up replays
+        g.replay()
+    torch.cuda.synchronize()
+    for lay, *_ in sets:
+        if lay.device_status() != 0:
+            raise SystemExit("device error flag set during warm-up")
+
+    def timed(g):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        return e0.elapsed_time(e1) / 1e3
+
+    with ClockSampler(local) as clk:
+        t_full = timed(g_full)
+    t_quant = timed(g_quant)
+    t_gemm = timed(g_gemm)
+    t_full_max = max_over_ranks(world, t_full)
+
+    # End-to-end through the host-buffer C ABI call: H2D of x, forward, D2H of y, sync.
+    layer, x, y, ws = sets[0]
+    xh = x.cpu().pin_memory()
+    yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        S.svdq_linear_forward_host(layer.handle, xh.data_ptr(), M, yh.data_ptr(), x.data_ptr(), y.data_ptr(),
+                                   ws.data_ptr(), stream)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        S.svdq_linear_forward_host(layer.handle, xh.data_ptr(), M, yh.data_ptr(), x.data_ptr(), y.data_ptr(),
+                                   ws.data_ptr(), stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = max_over_ranks(world, e0.elapsed_time(e1) / 1e3 / e2e_steps)
+    for lay, *_ in sets:
+        if lay.device_status() != 0:
+            raise SystemExit("device error flag set during the timed region")
+
+    fl = flops_per_step(M, K, N, R)
+    value = world * fl * args.steps / t_full_max / 1e12
+    pk = peaks()
+    fp4_peak = pk["bf16_tflops"] * FP4_PER_BF16
+    us_q = t_quant / args.steps * 1e6
+    us_g = t_gemm / args.steps * 1e6
+    q_gbs = quant_bytes(M, K, R) / (us_q * 1e-6) / 1e9
+    g_flops = 2.0 * M * N * K + 2.0 * M * N * R
+    g_tf = g_flops / (us_g * 1e-6) / 1e12
+    kernels = {
+        "quantize_act": {"us": us_q, "bound": "hbm", "algorithmic_bytes": quant_bytes(M, K, R),
+                         "achieved_gbs": q_gbs, "frac_of_hbm": q_gbs / pk["hbm_gbs"]},
+        "gemm_nvfp4_lr": {"us": us_g, "bound": "tensor", "algorithmic_flops": g_flops, "achieved_tflops": g_tf,
+                          "frac_of_fp4": g_tf / fp4_peak, "algorithmic_bytes": gemm_bytes(M, K, N, R),
+                          "achieved_gbs": gemm_bytes(M, K, N, R) / (us_g * 1e-6) / 1e9},
+    }
+    traffic = None
+    tf = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tf):
+        try:
+            with open(tf) as f:
+                traffic = json.load(f).get(ck.name, {}).get("gemm_nvfp4_lr")
+        except Exception:
+            traffic = None
+    if us_g >= us_q:
+        roof = {"kernel": "gemm_nvfp4_lr", "bound": "tensor", "achieved": g_tf, "peak": fp4_peak,
+                "unit": "TFLOP/s", "frac": g_tf / fp4_peak, "traffic": traffic,
+                "peak_source": f"{pk['source']} bf16 burst x {FP4_PER_BF16:g} (nominal FP4/BF16 ratio)"}
+    else:
+        roof = {"kernel": "quantize_act", "bound": "hbm", "achieved": q_gbs, "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": q_gbs / pk["hbm_gbs"], "traffic": None,
+                "peak_source": f"{pk['source']} copy bandwidth"}
+    step_us = t_full_max / args.steps * 1e6
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_us / 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4 (e2m1 x ue4m3/16) -> fp32 accumulate -> bf16", "data": "synthetic",
+        "config": config_of(ck),
+        "roofline": roof,
+        "roofline_step": {"bound": "tensor", "achieved": fl / (step_us * 1e-6) / 1e12, "peak": fp4_peak,
+                          "unit": "TFLOP/s", "frac": fl / (step_us * 1e-6) / 1e12 / fp4_peak},
+        "kernels": kernels,
+        "e2e": {"value": world * fl / t_e2e / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": 2 * M * K,
+                "d2h_bytes_per_step": 2 * M * N, "ms_per_step": t_e2e * 1e3,
+                "path": "svdq_linear_forward_host (pinned host x/y)"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = np.arange(min(M, args.ref_rows))
+        cpu_oracle_run(ck, rows[:16])
+        _, dt = cpu_oracle_run(ck, rows)
+        line["cpu_baseline"] = {"value": flops_per_step(len(rows), K, N, R) / dt / 1e12, "unit": "TFLOP/s",
+                                "cores": cpu_threads(), "kind": "oracle",
+                                "sample": f"{len(rows)} of {M} token rows of the workload, one run"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for lay, *_ in sets:
+        lay.close()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=None)
+    ap.add_argument("--ref-rows", type=int, default=1024)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    from bit_quantized_linear_svdq_b200 import synthetic
+    if args.workload is None:
+        args.workload = synthetic.HEADLINE
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup()
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

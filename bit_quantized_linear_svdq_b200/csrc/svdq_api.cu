@@ -1,0 +1,450 @@
+// svdq_api.cu -- the C ABI of include/svdq.h: argument checking, create-time
+// weight repacking into the layouts the kernels read, per-call tensor maps,
+// and the two launches of the forward pass.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/svdq.h"
+#include "kcommon.cuh"
+#include "svdq_kernels.h"
+
+struct svdq_linear {
+  int device;
+  int K, N, R, Kp, ka_pad, k_tiles, rotate_block;
+  uint8_t* qw;            // (N, Kp/2) packed E2M1, rows zero-padded to Kp
+  uint8_t* sfb;           // weight scale tiles: ceil(N/128) x ka_pad atoms of 512 bytes
+  __nv_bfloat16* pdT;     // proj_down^T (R, Kp), zero-padded
+  __nv_bfloat16* pu;      // proj_up (N, R)
+  float2* lam2;           // (Kp) {smooth, 1/smooth}, padded with {1, 1}
+  float* alpha;           // (roundup(N, 128)) wcscales * wtscale, zero-padded
+  unsigned* err;          // device error word
+  CUtensorMap tm_b, tm_pdT, tm_pu;
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+svdq_status cuda_fail(cudaError_t e, const char* where) {
+  g_last_error = std::string(where) + ": " + cudaGetErrorString(e);
+  return SVDQ_ERR_CUDA;
+}
+
+#define SVDQ_CUDA(call)                                        \
+  do {                                                         \
+    cudaError_t e_ = (call);                                   \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call);        \
+  } while (0)
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor map with the 128-byte swizzle; out-of-bounds reads are zero.
+svdq_status make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+                      uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    g_last_error = "cuTensorMapEncodeTiled unavailable";
+    return SVDQ_ERR_CUDA;
+  }
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_last_error = "cuTensorMapEncodeTiled failed with CUresult " + std::to_string((int)r);
+    return SVDQ_ERR_CUDA;
+  }
+  return SVDQ_OK;
+}
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- create-time repack kernels
+
+__global__ void repack_weight_scales(const uint8_t* __restrict__ wscales, uint8_t* __restrict__ sfb, int K16, int N,
+                                     int ka_pad, unsigned* bad) {
+  const long long total = (long long)K16 * N;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
+    const int kb = (int)(i / N), n = (int)(i % N);
+    const uint8_t b = wscales[i];
+    if ((b & 0x7F) == 0x7F) atomicOr(bad, 1u);       // e4m3 NaN
+    sfb[((size_t)(n >> 7) * ka_pad + (kb >> 2)) * svdq::kSfAtomBytes + svdq::sf_atom_offset(n & 127, kb & 3)] = b;
+  }
+}
+
+__global__ void transpose_proj_down(const __nv_bfloat16* __restrict__ pd, __nv_bfloat16* __restrict__ pdT, int K,
+                                    int R, int Kp) {
+  const long long total = (long long)R * Kp;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(i / Kp), k = (int)(i % Kp);
+    pdT[i] = k < K ? pd[(size_t)k * R + r] : __float2bfloat16_rn(0.0f);
+  }
+}
+
+__global__ void prepare_smooth(const __nv_bfloat16* __restrict__ sf, float2* __restrict__ lam2, int K, int Kp,
+                               unsigned* bad) {
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < Kp; k += gridDim.x * blockDim.x) {
+    if (k < K) {
+      const float l = __bfloat162float(sf[k]);
+      if (!(isfinite(l) && l != 0.0f)) atomicOr(bad, 2u);
+      lam2[k] = make_float2(l, __frcp_rn(l));
+    } else {
+      lam2[k] = make_float2(1.0f, 1.0f);
+    }
+  }
+}
+
+__global__ void prepare_alpha(const __nv_bfloat16* __restrict__ wc, const __nv_bfloat16* __restrict__ wt, float* alpha,
+                              int N, int Npad) {
+  const float t = wt ? __bfloat162float(wt[0]) : 1.0f;
+  for (int n = blockIdx.x * blockDim.x + threadIdx.x; n < Npad; n += gridDim.x * blockDim.x) {
+    // bf16 x bf16 is exact in fp32.
+    alpha[n] = n < N ? (wc ? __bfloat162float(wc[n]) : 1.0f) * t : 0.0f;
+  }
+}
+
+int grid_for(long long n) {
+  long long g = (n + 255) / 256;
+  return (int)(g < 1 ? 1 : (g > 4096 ? 4096 : g));
+}
+
+svdq_status check_device(const svdq_linear* h) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev != h->device) {
+    g_last_error = "current device differs from the device the handle was created on";
+    return SVDQ_ERR_INVALID_ARG;
+  }
+  return SVDQ_OK;
+}
+
+void free_handle(svdq_linear* h) {
+  if (!h) return;
+  cudaFree(h->qw);
+  cudaFree(h->sfb);
+  cudaFree(h->pdT);
+  cudaFree(h->pu);
+  cudaFree(h->lam2);
+  cudaFree(h->alpha);
+  cudaFree(h->err);
+  delete h;
+}
+
+struct WsLayout {
+  size_t codes, sfa, lr, total;
+};
+
+WsLayout ws_layout(const svdq_linear* h, int M) {
+  WsLayout w;
+  w.codes = 0;
+  w.sfa = align256((size_t)M * (h->Kp / 2));
+  w.lr = align256(w.sfa + (size_t)((M + 127) / 128) * h->ka_pad * svdq::kSfAtomBytes);
+  w.total = align256(w.lr + (size_t)M * h->R * 2);
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+int svdq_version(void) { return (1 << 16) | 0; }
+
+const char* svdq_status_string(svdq_status s) {
+  switch (s) {
+    case SVDQ_OK: return "ok";
+    case SVDQ_ERR_INVALID_ARG: return "invalid argument";
+    case SVDQ_ERR_SHAPE: return "unsupported shape";
+    case SVDQ_ERR_UNSUPPORTED: return "unsupported device or configuration";
+    case SVDQ_ERR_CUDA: return "CUDA error";
+    case SVDQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case SVDQ_ERR_DEVICE: return "device-side error (bounded wait expired)";
+  }
+  return "unknown status";
+}
+
+const char* svdq_last_error(void) { return g_last_error.c_str(); }
+
+svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, void* stream_) {
+  if (!out) return SVDQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!d || !d->qweight || !d->wscales || !d->proj_down || !d->proj_up || !d->smooth_factor)
+    return SVDQ_ERR_INVALID_ARG;
+  if (d->act_unsigned != 0) return SVDQ_ERR_UNSUPPORTED;
+  if (d->K <= 0 || d->N <= 0 || d->K % 16 != 0) return SVDQ_ERR_SHAPE;
+  if (d->R < 16 || d->R > 128 || d->R % 16 != 0) return SVDQ_ERR_SHAPE;
+  if (d->rotate_block != 0 && d->rotate_block != 128) return SVDQ_ERR_SHAPE;
+  if (d->rotate_block && d->K % d->rotate_block != 0) return SVDQ_ERR_SHAPE;
+  if ((long long)d->K * d->N > (1LL << 40)) return SVDQ_ERR_SHAPE;
+
+  int dev = 0, major = 0, minor = 0;
+  SVDQ_CUDA(cudaGetDevice(&dev));
+  SVDQ_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  SVDQ_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+  if (major != 10 || minor != 0) {
+    g_last_error = "requires an sm_100 (B200) device";
+    return SVDQ_ERR_UNSUPPORTED;
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+
+  svdq_linear* h = new svdq_linear();
+  std::memset(h, 0, sizeof(*h));
+  h->device = dev;
+  h->K = d->K;
+  h->N = d->N;
+  h->R = d->R;
+  h->rotate_block = d->rotate_block;
+  h->Kp = (d->K + 127) / 128 * 128;
+  h->k_tiles = (h->Kp + 255) / 256;
+  h->ka_pad = 4 * h->k_tiles;
+  const int n_tiles = (d->N + 127) / 128;
+  const int Npad = n_tiles * 128;
+
+  auto fail = [&](svdq_status s) {
+    free_handle(h);
+    return s;
+  };
+  cudaError_t e;
+#define CREATE_CUDA(call)                         \
+  do {                                            \
+    e = (call);                                   \
+    if (e != cudaSuccess) {                       \
+      cuda_fail(e, #call);                        \
+      return fail(SVDQ_ERR_CUDA);                 \
+    }                                             \
+  } while (0)
+
+  CREATE_CUDA(cudaMalloc(&h->qw, (size_t)d->N * (h->Kp / 2)));
+  CREATE_CUDA(cudaMalloc(&h->sfb, (size_t)n_tiles * h->ka_pad * svdq::kSfAtomBytes));
+  CREATE_CUDA(cudaMalloc(&h->pdT, (size_t)d->R * h->Kp * 2));
+  CREATE_CUDA(cudaMalloc(&h->pu, (size_t)d->N * d->R * 2));
+  CREATE_CUDA(cudaMalloc(&h->lam2, (size_t)h->Kp * sizeof(float2)));
+  CREATE_CUDA(cudaMalloc(&h->alpha, (size_t)Npad * sizeof(float)));
+  CREATE_CUDA(cudaMalloc(&h->err, 2 * sizeof(unsigned)));   // [0] device error word, [1] create-time checks
+  CREATE_CUDA(cudaMemsetAsync(h->err, 0, 2 * sizeof(unsigned), stream));
+
+  CREATE_CUDA(cudaMemset2DAsync(h->qw, h->Kp / 2, 0, h->Kp / 2, d->N, stream));
+  CREATE_CUDA(cudaMemcpy2DAsync(h->qw, h->Kp / 2, d->qweight, d->K / 2, d->K / 2, d->N, cudaMemcpyDeviceToDevice,
+                                stream));
+  CREATE_CUDA(cudaMemsetAsync(h->sfb, 0, (size_t)n_tiles * h->ka_pad * svdq::kSfAtomBytes, stream));
+  repack_weight_scales<<<grid_for((long long)(d->K / 16) * d->N), 256, 0, stream>>>(
+      static_cast<const uint8_t*>(d->wscales), h->sfb, d->K / 16, d->N, h->ka_pad, h->err + 1);
+  CREATE_CUDA(cudaGetLastError());
+  transpose_proj_down<<<grid_for((long long)d->R * h->Kp), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(d->proj_down), h->pdT, d->K, d->R, h->Kp);
+  CREATE_CUDA(cudaGetLastError());
+  CREATE_CUDA(cudaMemcpyAsync(h->pu, d->proj_up, (size_t)d->N * d->R * 2, cudaMemcpyDeviceToDevice, stream));
+  prepare_smooth<<<grid_for(h->Kp), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(d->smooth_factor), h->lam2,
+                                                       d->K, h->Kp, h->err + 1);
+  CREATE_CUDA(cudaGetLastError());
+  prepare_alpha<<<grid_for(Npad), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(d->wcscales),
+                                                     static_cast<const __nv_bfloat16*>(d->wtscale), h->alpha, d->N,
+                                                     Npad);
+  CREATE_CUDA(cudaGetLastError());
+  unsigned bad = 0;
+  CREATE_CUDA(cudaMemcpyAsync(&bad, h->err + 1, sizeof(unsigned), cudaMemcpyDeviceToHost, stream));
+  CREATE_CUDA(cudaStreamSynchronize(stream));
+  if (bad) {
+    g_last_error = (bad & 1u) ? "wscales holds an e4m3 NaN" : "smooth_factor holds a zero or non-finite value";
+    return fail(SVDQ_ERR_INVALID_ARG);
+  }
+#undef CREATE_CUDA
+
+  svdq_status s;
+  if ((s = make_tmap(&h->tm_b, h->qw, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->Kp / 2, d->N, h->Kp / 2, 128, 128)) != SVDQ_OK)
+    return fail(s);
+  if ((s = make_tmap(&h->tm_pdT, h->pdT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->Kp, d->R, (uint64_t)h->Kp * 2, 64,
+                     d->R)) != SVDQ_OK)
+    return fail(s);
+  if ((s = make_tmap(&h->tm_pu, h->pu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d->R, d->N, (uint64_t)d->R * 2, 64, 128)) !=
+      SVDQ_OK)
+    return fail(s);
+  *out = h;
+  return SVDQ_OK;
+}
+
+void svdq_linear_destroy(svdq_linear* h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  free_handle(h);
+}
+
+size_t svdq_workspace_bytes(const svdq_linear* h, int M) {
+  if (!h || M <= 0) return 0;
+  return ws_layout(h, M).total;
+}
+
+svdq_status svdq_quantize_act(const svdq_linear* h, const void* x, int M, void* codes, void* scales, void* lowrank,
+                              void* stream_) {
+  if (!h || M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!x || !codes || !scales) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || (lowrank && !aligned16(lowrank))) return SVDQ_ERR_INVALID_ARG;
+  svdq_status s = check_device(h);
+  if (s != SVDQ_OK) return s;
+  svdq::QuantLaunch q;
+  if ((s = make_tmap(&q.tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->K, M, (uint64_t)h->K * 2, 64, 128)) != SVDQ_OK)
+    return s;
+  q.tm_pdT = h->tm_pdT;
+  q.lam2 = h->lam2;
+  q.codes = static_cast<uint8_t*>(codes);
+  q.scales = static_cast<uint8_t*>(scales);
+  q.lowrank = lowrank;
+  q.err = h->err;
+  q.M = M;
+  q.K = h->K;
+  q.Kp = h->Kp;
+  q.R = h->R;
+  q.codes_pitch = h->K / 2;
+  q.scales_pitch = h->K / 16;
+  q.k_limit = h->K;
+  q.ka_pad = h->ka_pad;
+  q.tiled_scales = false;
+  q.rotate_block = h->rotate_block;
+  cudaError_t e = svdq::launch_quantize_act(q, static_cast<cudaStream_t>(stream_));
+  if (e != cudaSuccess) return cuda_fail(e, "quantize_act launch");
+  return SVDQ_OK;
+}
+
+namespace {
+
+svdq_status check_forward_args(const svdq_linear* h, int M, void* workspace) {
+  if (!h || M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SVDQ_ERR_WORKSPACE;
+  return check_device(h);
+}
+
+svdq_status forward_quantize(const svdq_linear* h, const void* x, int M, void* workspace, cudaStream_t stream) {
+  const WsLayout w = ws_layout(h, M);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  svdq::QuantLaunch q;
+  svdq_status s;
+  if ((s = make_tmap(&q.tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->K, M, (uint64_t)h->K * 2, 64, 128)) != SVDQ_OK)
+    return s;
+  q.tm_pdT = h->tm_pdT;
+  q.lam2 = h->lam2;
+  q.codes = ws + w.codes;
+  q.scales = ws + w.sfa;
+  q.lowrank = ws + w.lr;
+  q.err = h->err;
+  q.M = M;
+  q.K = h->K;
+  q.Kp = h->Kp;
+  q.R = h->R;
+  q.codes_pitch = h->Kp / 2;
+  q.scales_pitch = 0;
+  q.k_limit = h->Kp;
+  q.ka_pad = h->ka_pad;
+  q.tiled_scales = true;
+  q.rotate_block = h->rotate_block;
+  cudaError_t e = svdq::launch_quantize_act(q, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "quantize_act launch");
+  return SVDQ_OK;
+}
+
+svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, cudaStream_t stream) {
+  const WsLayout w = ws_layout(h, M);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  svdq::GemmLaunch g;
+  svdq_status s;
+  if ((s = make_tmap(&g.tm_a, ws + w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->Kp / 2, M, h->Kp / 2, 128, 128)) !=
+      SVDQ_OK)
+    return s;
+  g.tm_b = h->tm_b;
+  if ((s = make_tmap(&g.tm_l, ws + w.lr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->R, M, (uint64_t)h->R * 2, 64, 128)) !=
+      SVDQ_OK)
+    return s;
+  g.tm_pu = h->tm_pu;
+  g.sfa = ws + w.sfa;
+  g.sfb = h->sfb;
+  g.alpha = h->alpha;
+  g.y = y;
+  g.err = h->err;
+  g.M = M;
+  g.N = h->N;
+  g.R = h->R;
+  g.k_tiles = h->k_tiles;
+  g.ka_pad = h->ka_pad;
+  cudaError_t e = svdq::launch_gemm_nvfp4_lr(g, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+  return SVDQ_OK;
+}
+
+}  // namespace
+
+svdq_status svdq_linear_forward_quantize(const svdq_linear* h, const void* x, int M, void* workspace, void* stream) {
+  svdq_status s = check_forward_args(h, M, workspace);
+  if (s != SVDQ_OK || M == 0) return s;
+  if (!x || !aligned16(x)) return SVDQ_ERR_INVALID_ARG;
+  return forward_quantize(h, x, M, workspace, static_cast<cudaStream_t>(stream));
+}
+
+svdq_status svdq_linear_forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, void* stream) {
+  svdq_status s = check_forward_args(h, M, workspace);
+  if (s != SVDQ_OK || M == 0) return s;
+  if (!y || !aligned16(y)) return SVDQ_ERR_INVALID_ARG;
+  return forward_gemm(h, M, y, workspace, static_cast<cudaStream_t>(stream));
+}
+
+svdq_status svdq_linear_forward(const svdq_linear* h, const void* x, int M, void* y, void* workspace, void* stream_) {
+  if (!h || M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!x || !y || !aligned16(x) || !aligned16(y)) return SVDQ_ERR_INVALID_ARG;
+  svdq_status s = check_forward_args(h, M, workspace);
+  if (s != SVDQ_OK) return s;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if ((s = forward_quantize(h, x, M, workspace, stream)) != SVDQ_OK) return s;
+  return forward_gemm(h, M, y, workspace, stream);
+}
+
+svdq_status svdq_linear_forward_host(const svdq_linear* h, const void* x_host, int M, void* y_host, void* x_dev,
+                                     void* y_dev, void* workspace, void* stream_) {
+  if (!h || M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!x_host || !y_host) return SVDQ_ERR_INVALID_ARG;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  SVDQ_CUDA(cudaMemcpyAsync(x_dev, x_host, (size_t)M * h->K * 2, cudaMemcpyHostToDevice, stream));
+  svdq_status s = svdq_linear_forward(h, x_dev, M, y_dev, workspace, stream_);
+  if (s != SVDQ_OK) return s;
+  SVDQ_CUDA(cudaMemcpyAsync(y_host, y_dev, (size_t)M * h->N * 2, cudaMemcpyDeviceToHost, stream));
+  SVDQ_CUDA(cudaStreamSynchronize(stream));
+  return SVDQ_OK;
+}
+
+svdq_status svdq_device_status(const svdq_linear* h, int* flags) {
+  if (!h) return SVDQ_ERR_INVALID_ARG;
+  svdq_status s = check_device(h);
+  if (s != SVDQ_OK) return s;
+  SVDQ_CUDA(cudaDeviceSynchronize());
+  unsigned v = 0;
+  SVDQ_CUDA(cudaMemcpy(&v, h->err, sizeof(unsigned), cudaMemcpyDeviceToHost));
+  if (v) SVDQ_CUDA(cudaMemset(h->err, 0, sizeof(unsigned)));
+  if (flags) *flags = (int)v;
+  return v ? SVDQ_ERR_DEVICE : SVDQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,49 @@
+// svdq_kernels.h -- host-side launch interface of the two hot-path kernels
+// (internal to the library; the public boundary is include/svdq.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace svdq {
+
+// Fused activation quantizer: x_hat = x / smooth (optionally block-Hadamard
+// rotated), NVFP4 codes + e4m3 scales, and L = x_hat @ proj_down.
+struct QuantLaunch {
+  CUtensorMap tm_x;         // x bf16 (M, K): box {64, 128}, 128B swizzle
+  CUtensorMap tm_pdT;       // proj_down^T bf16 (R, Kp): box {64, R}, 128B swizzle
+  const void* lam2;         // float2 (Kp): {smooth, 1/smooth}, padded with {1, 1}
+  uint8_t* codes;           // packed codes, row pitch codes_pitch bytes
+  uint8_t* scales;          // row-major (pitch scales_pitch) or tensor-core tiles
+  void* lowrank;            // bf16 (M, R) or nullptr
+  unsigned* err;            // device error word
+  int M, K, Kp, R;
+  int codes_pitch;          // bytes per row of codes
+  int scales_pitch;         // bytes per row of row-major scales
+  int k_limit;              // codes/scales are written for k < k_limit only
+  int ka_pad;               // tiled scales: 64-element K atoms per 128-row tile
+  bool tiled_scales;        // scale layout: tensor-core tiles instead of row-major
+  int rotate_block;         // 0 or 128
+};
+cudaError_t launch_quantize_act(const QuantLaunch& p, cudaStream_t stream);
+
+// Block-scaled NVFP4 GEMM with the rank-R up-projection and the
+// wcscales * wtscale scaling fused into the epilogue.
+struct GemmLaunch {
+  CUtensorMap tm_a;         // activation codes u8 (M, Kp/2): box {128, 128}, 128B swizzle
+  CUtensorMap tm_b;         // weight codes u8 (N, Kp/2): box {128, 128}, 128B swizzle
+  CUtensorMap tm_l;         // L bf16 (M, R): box {64, 128}, 128B swizzle
+  CUtensorMap tm_pu;        // proj_up bf16 (N, R): box {64, 128}, 128B swizzle
+  const uint8_t* sfa;       // activation scale tiles
+  const uint8_t* sfb;       // weight scale tiles
+  const float* alpha;       // (N padded to 128) wcscales * wtscale
+  void* y;                  // bf16 (M, N)
+  unsigned* err;
+  int M, N, R;
+  int k_tiles;              // Kp rounded up to 256, divided by 256
+  int ka_pad;               // K atoms per 128-row scale tile (= 4 * k_tiles)
+};
+cudaError_t launch_gemm_nvfp4_lr(const GemmLaunch& p, cudaStream_t stream);
+
+}  // namespace svdq

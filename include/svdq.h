@@ -1,0 +1,176 @@
+/*
+ * svdq.h -- C ABI of the B200 (sm_100a) SVDQuant W4A4 linear layer.
+ *
+ * The layer ("SVDQuant W4A4", vLLM-Omni svdquant.md, sections "Overview",
+ * "Checkpoint contract", "Runtime support") computes, for bf16 activations
+ * x[M, K] and an offline-quantized checkpoint,
+ *
+ *   x_hat = x / smooth_factor                      (per input channel k)
+ *   x_hat = x_hat R^T   (optional: R = blockdiag(H_128 / sqrt(128)), the
+ *                        normalized Sylvester Hadamard of "Rotate in
+ *                        quantization and its vLLM implementation",
+ *                        sections 2.1-2.2; the weight was rotated offline)
+ *   y     = wcscales (.) wtscale * (Q(x_hat) Q(W)^T) + (x_hat proj_down) proj_up^T
+ *
+ * in bf16, where Q() is NVFP4: E2M1 codes {0,.5,1,1.5,2,3,4,6} x sign, two
+ * per byte (element 2j in the low nibble of byte j), one e4m3 (OCP FP8
+ * E4M3FN) scale per 16 consecutive K elements.  Activations are quantized
+ * online with scale = e4m3_rne_satfinite(fp32(amax/6)) and
+ * code = e2m1_rne_satfinite(fp32(x_hat / scale)) (a block whose scale rounds
+ * to zero gets scale 0 and codes 0).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers (cudaMalloc'd or otherwise
+ *    device-accessible) unless a name ends in _host.  All tensors are dense,
+ *    row-major, with no padding between rows.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued asynchronously on it; nothing synchronizes unless stated.
+ *  - Functions return an svdq_status and never throw across the ABI.  On
+ *    SVDQ_ERR_CUDA the CUDA error text is available from svdq_last_error().
+ *  - The device must be compute capability 10.0 (B200, sm_100a); create()
+ *    checks the current device.
+ *  - A handle is used on the device that was current at create().  Calls on
+ *    one handle from several host threads are safe (the handle is read-only
+ *    after create) as long as their workspaces differ.
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SVDQ_API __attribute__((visibility("default")))
+#else
+#define SVDQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,   /* null pointer, bad flag, misaligned pointer, M < 0 */
+  SVDQ_ERR_SHAPE = 2,         /* K % 16 != 0, R not in {16..128} step 16, rotate block does not divide K */
+  SVDQ_ERR_UNSUPPORTED = 3,   /* not an sm_100 device, act_unsigned != 0, precision other than nvfp4 */
+  SVDQ_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed (see svdq_last_error) */
+  SVDQ_ERR_WORKSPACE = 5,     /* workspace NULL or too small for M */
+  SVDQ_ERR_DEVICE = 6         /* a kernel reported a device-side error (bounded wait expired) */
+} svdq_status;
+
+/* Opaque handle: library-owned, repacked copies of one layer's weights. */
+typedef struct svdq_linear svdq_linear;
+
+/*
+ * Layer description at create time.  Shapes and dtypes are the checkpoint
+ * contract of "SVDQuant W4A4" (section "Checkpoint contract"); K must be a
+ * multiple of 16 (same section).  The library reads rank / precision /
+ * act_unsigned of the checkpoint's quantization_config through K, N, R and
+ * act_unsigned; precision is always "nvfp4".
+ */
+typedef struct {
+  int K;                      /* input features, multiple of 16 (and of rotate_block if set) */
+  int N;                      /* output features, >= 1 */
+  int R;                      /* low-rank correction rank: 16, 32, ..., 128 */
+  int rotate_block;           /* 0 = no online rotation, 128 = block Hadamard of size 128 */
+  int act_unsigned;           /* must be 0 (signed activations) */
+  const void* qweight;        /* (N, K/2)  int8: packed E2M1, element 2j in low nibble of byte j */
+  const void* wscales;        /* (K/16, N) float8_e4m3fn: wscales[k/16, n] scales W[n, k] */
+  const void* proj_down;      /* (K, R)    bf16 */
+  const void* proj_up;        /* (N, R)    bf16 */
+  const void* smooth_factor;  /* (K,)      bf16, finite and nonzero */
+  const void* wcscales;       /* (N,)      bf16, or NULL meaning all ones */
+  const void* wtscale;        /* (1,)      bf16, or NULL meaning 1.0 */
+} svdq_linear_desc;
+
+/*
+ * svdq_linear_create -- validate the description and copy + repack the
+ * weights into library-owned device memory (FP4 weight rows padded for TMA,
+ * scale factors re-tiled into the tensor-core scale layout, proj_down
+ * transposed, alpha[n] = wcscales[n] * wtscale precomputed in fp32).
+ * The source tensors may be freed once this returns: it synchronizes `stream`.
+ * On success *out receives the handle; on failure *out is set to NULL.
+ * Shape errors are reported here (the pages' fail-at-load convention,
+ * "SVDQuant W4A4" section "Runtime support").
+ */
+SVDQ_API svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* desc, void* stream);
+
+/* Free the handle and its device memory.  NULL is a no-op.  Synchronizes the device. */
+SVDQ_API void svdq_linear_destroy(svdq_linear* h);
+
+/* Bytes of device workspace svdq_linear_forward needs for M rows (0 for M == 0). */
+SVDQ_API size_t svdq_workspace_bytes(const svdq_linear* h, int M);
+
+/*
+ * svdq_quantize_act -- the fused activation quantizer alone (smooth, optional
+ * rotation, NVFP4 quantize, and the rank-R down-projection from the same read
+ * of x).
+ *   x       (M, K)    bf16, input
+ *   codes   (M, K/2)  uint8 output: packed E2M1 codes, low nibble = even k
+ *   scales  (M, K/16) uint8 output: e4m3 scale bytes, row-major
+ *   lowrank (M, R)    bf16 output L = x_hat proj_down (fp32 accumulate of
+ *                     bf16(x_hat) products), or NULL to skip writing it
+ * M == 0 is a no-op.  Pointers must be 16-byte aligned.
+ */
+SVDQ_API svdq_status svdq_quantize_act(const svdq_linear* h, const void* x, int M,
+                              void* codes, void* scales, void* lowrank, void* stream);
+
+/*
+ * svdq_linear_forward -- y (M, N) bf16 = the full layer on x (M, K) bf16.
+ * Two kernels on `stream`: the fused quantizer (writes codes, tensor-core
+ * scale tiles and L into `workspace`) and the block-scaled FP4 GEMM whose
+ * epilogue adds the rank-R up-projection and applies wcscales * wtscale.
+ * workspace: >= svdq_workspace_bytes(h, M) bytes of device memory, 256-byte
+ * aligned, owned by the caller, not shared by concurrent calls.
+ */
+SVDQ_API svdq_status svdq_linear_forward(const svdq_linear* h, const void* x, int M, void* y,
+                                void* workspace, void* stream);
+
+/*
+ * The two stages of svdq_linear_forward, callable separately (same
+ * arguments; together they are exactly svdq_linear_forward):
+ *   svdq_linear_forward_quantize -- the fused quantizer: x -> codes, scale
+ *       tiles and L inside `workspace`.
+ *   svdq_linear_forward_gemm     -- the GEMM + rank-R epilogue: workspace -> y.
+ * The workspace written by the first call must be passed unchanged, with the
+ * same M, to the second; stream order between them is the caller's.
+ */
+SVDQ_API svdq_status svdq_linear_forward_quantize(const svdq_linear* h, const void* x, int M,
+                                                  void* workspace, void* stream);
+SVDQ_API svdq_status svdq_linear_forward_gemm(const svdq_linear* h, int M, void* y,
+                                              void* workspace, void* stream);
+
+/*
+ * svdq_linear_forward_host -- end-to-end call on HOST buffers: copies x_host
+ * (M, K bf16) to x_dev, runs svdq_linear_forward into y_dev, copies y_dev to
+ * y_host (M, N bf16) and synchronizes `stream` before returning.  Host
+ * buffers should be pinned for full copy bandwidth.  x_dev / y_dev /
+ * workspace are caller-owned device buffers as in svdq_linear_forward.
+ */
+SVDQ_API svdq_status svdq_linear_forward_host(const svdq_linear* h, const void* x_host, int M, void* y_host,
+                                     void* x_dev, void* y_dev, void* workspace, void* stream);
+
+/*
+ * svdq_device_status -- synchronize the handle's device and read + clear its
+ * device error word (nonzero when a kernel's bounded wait expired: the kernel
+ * then skipped its remaining work, released its tensor memory and returned).
+ * *flags receives the word (bit 0: quantizer, bit 1: GEMM).  Returns
+ * SVDQ_ERR_DEVICE when it was nonzero.
+ */
+SVDQ_API svdq_status svdq_device_status(const svdq_linear* h, int* flags);
+
+/* Static text for a status code. */
+SVDQ_API const char* svdq_status_string(svdq_status s);
+
+/* Text of the last CUDA error seen by this thread ("" if none). */
+SVDQ_API const char* svdq_last_error(void);
+
+/* ABI version: (major << 16) | minor. */
+SVDQ_API int svdq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H_ */

@@ -1,0 +1,74 @@
+"""C-ABI checks that need no GPU: the library builds and loads, it exports
+every entry point include/svdq.h declares, and host-side argument validation
+answers before any device work."""
+import ctypes
+
+import pytest
+
+import bit_quantized_linear_svdq_b200 as S
+from bit_quantized_linear_svdq_b200 import build as B
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return S.load_library()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = S.exported_names()
+    assert set(names) == {
+        "svdq_linear_create", "svdq_linear_destroy", "svdq_workspace_bytes", "svdq_quantize_act",
+        "svdq_linear_forward", "svdq_linear_forward_host", "svdq_device_status", "svdq_status_string",
+        "svdq_last_error", "svdq_version", "svdq_linear_forward_quantize", "svdq_linear_forward_gemm"}
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings_and_version(lib):
+    assert S.svdq_version() >> 16 == 1
+    for code in range(7):
+        assert S.svdq_status_string(code)
+    assert S.svdq_status_string(0) == "ok"
+
+
+def _desc(**kw):
+    base = dict(K=256, N=256, R=32, rotate_block=0, act_unsigned=0, qweight=1, wscales=1, proj_down=1,
+                proj_up=1, smooth_factor=1, wcscales=None, wtscale=None)
+    base.update(kw)
+    return S.svdq_linear_desc(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(K=24), 2),                 # K % 16
+    (dict(K=0), 2),
+    (dict(N=0), 2),
+    (dict(R=8), 2),
+    (dict(R=40), 2),
+    (dict(R=256), 2),
+    (dict(rotate_block=64), 2),
+    (dict(K=272, rotate_block=128), 2),
+    (dict(act_unsigned=1), 3),
+    (dict(qweight=None), 1),
+    (dict(smooth_factor=None), 1),
+])
+def test_create_validation_is_host_side(lib, kw, status):
+    h = ctypes.c_void_p(123)
+    st = lib.svdq_linear_create(ctypes.byref(h), ctypes.byref(_desc(**kw)), None)
+    assert st == status
+    assert h.value is None
+
+
+def test_null_handle_calls(lib):
+    assert lib.svdq_workspace_bytes(None, 16) == 0
+    assert lib.svdq_quantize_act(None, 1, 1, 1, 1, None, None) == 1
+    assert lib.svdq_linear_forward(None, 1, 1, 1, 1, None) == 1
+    assert lib.svdq_linear_create(None, None, None) == 1
+    lib.svdq_linear_destroy(None)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(S, "_lib", None)
+    monkeypatch.setattr(S, "library_path", lambda: str(tmp_path / "nope.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        S.load_library()

@@ -1,0 +1,252 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.
+
+Bars (from the layer's definition and its NVFP4 conventions):
+  * packed E2M1 codes and e4m3 scale bytes: bit-exact;
+  * y (bf16): relative Frobenius error <= 5e-3 and every element within
+    1e-2 * max|y_oracle|;
+  * L = x_hat @ proj_down (bf16, from bf16(x_hat) on tensor cores): relative
+    Frobenius error <= 1e-2 (two bf16 roundings of ~2^-9 each, see design notes).
+"""
+import numpy as np
+import pytest
+import torch
+
+import bit_quantized_linear_svdq_b200 as S
+from bit_quantized_linear_svdq_b200 import synthetic
+from oracle import svdq_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+Y_REL_FRO = 5e-3
+Y_MAX_REL = 1e-2
+L_REL_FRO = 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from bit_quantized_linear_svdq_b200 import build
+    build.build()
+    S.load_library()
+
+
+def dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def dev_u8(a):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.uint8)).cuda()
+
+
+def host_bf16_to_f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def weights_of(ck):
+    if ck.qweight is None:
+        qw, ws = O.quantize_weight_nvfp4(ck.dense_weight, ck.rotate_block)
+        ck.qweight, ck.wscales = qw, ws
+    return ck
+
+
+def make_layer(ck, with_wc=True):
+    ck = weights_of(ck)
+    return S.SVDQLinear(dev_u8(ck.qweight), dev_u8(ck.wscales), dev_bf16(ck.proj_down), dev_bf16(ck.proj_up),
+                        dev_bf16(ck.smooth_factor), dev_bf16(ck.wcscales) if with_wc else None,
+                        dev_bf16(ck.wtscale) if with_wc else None, rotate_block=ck.rotate_block)
+
+
+def assert_y_close(y_gpu, y_ref, what=""):
+    err = y_gpu - y_ref
+    rel = np.linalg.norm(err) / max(np.linalg.norm(y_ref), 1e-30)
+    mx = np.max(np.abs(err)) / max(np.max(np.abs(y_ref)), 1e-30)
+    assert rel <= Y_REL_FRO, f"{what} rel-Frobenius {rel:.3e}"
+    assert mx <= Y_MAX_REL, f"{what} max-abs/max|y| {mx:.3e}"
+
+
+def check_quantizer(layer, ck, rows=None):
+    x = dev_bf16(ck.x)
+    codes, scales, lowrank = layer.quantize_act(x)
+    torch.cuda.synchronize()
+    xb = ck.x if rows is None else ck.x[rows]
+    c_ref, s_ref, xh = O.quantize_act(xb, ck.smooth_factor, ck.rotate_block)
+    c_gpu = codes.cpu().numpy()
+    s_gpu = scales.cpu().numpy()
+    if rows is not None:
+        c_gpu, s_gpu = c_gpu[rows], s_gpu[rows]
+    np.testing.assert_array_equal(s_gpu, s_ref)
+    bad = np.argwhere(c_gpu != c_ref)
+    assert bad.size == 0, f"{len(bad)} code bytes differ, first at {bad[:5].tolist()}"
+    L_ref = O.lowrank_down(xh, ck.proj_down)
+    L_gpu = host_bf16_to_f64(lowrank)
+    if rows is not None:
+        L_gpu = L_gpu[rows]
+    rel = np.linalg.norm(L_gpu - L_ref) / max(np.linalg.norm(L_ref), 1e-30)
+    assert rel <= L_REL_FRO, f"L rel-Frobenius {rel:.3e}"
+
+
+def check_forward(layer, ck, rows=None):
+    x = dev_bf16(ck.x)
+    y = layer.forward(x)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    y_gpu = host_bf16_to_f64(y)
+    if rows is not None:
+        y_gpu = y_gpu[rows]
+    y_ref = O.linear_forward(ck, rows=rows)
+    assert_y_close(y_gpu, y_ref, ck.name)
+    return y
+
+
+# ------------------------------------------------------------------ number-format semantics
+
+def test_convert_semantics_ties_signed_zero_saturation():
+    """Hand-made blocks exercising ties-to-even, negative values rounding to
+    zero (sign kept), scale saturation and zero / tiny blocks."""
+    K = 64
+    rows = []
+    mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    r0 = [6.0] + mids + [-m for m in mids] + [0.0]
+    rows.append(r0 + [-6.0] + [-m for m in mids] + mids + [0.0] + [0.0] * 32)
+    rows.append([6.0, -0.1, -0.2, 0.1, 0.24, -0.24, 0.26, -0.26] + [0.0] * 8 + [1e4] + [1.0] * 15 + [0.0] * 32)
+    rows.append([0.0] * 16 + [1e-4] * 16 + [-3e-3] + [0.0] * 15 + [448.0 * 6] + [-1.0] * 15)
+    rows.append([float(v) for v in np.linspace(-7, 7, K)])
+    x = np.array(rows, dtype=np.float32)
+    bits = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    ck = synthetic.make_checkpoint(4, K, 16, 16, seed=0, n_outliers=0)
+    ck.x = bits
+    ck.smooth_factor = torch.ones(K).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    layer = make_layer(ck)
+    check_quantizer(layer, ck)
+    check_forward(layer, ck)
+
+
+# ------------------------------------------------------------------ the named workloads
+
+SMALL = ["tiny_16x256x256_r32"]
+FULL = ["attn_proj_4096x3072x3072_r32", "mlp_up_4096x3072x12288_r32", "mlp_down_rot128_4096x12288x3072_r32",
+        "small_batch_m1_4096x4096_r32", "small_batch_m16_4096x4096_r32", "small_batch_m64_4096x4096_r32",
+        "small_batch_m256_4096x4096_r32", "small_batch_m1024_4096x4096_r32",
+        "rank_sweep_4096x3072x3072_r16", "rank_sweep_4096x3072x3072_r64", "rank_sweep_4096x3072x3072_r128"]
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_small_workload_full_parity(name):
+    ck = synthetic.load(name)
+    layer = make_layer(ck)
+    check_quantizer(layer, ck)
+    check_forward(layer, ck)
+
+
+def _sample_rows(M, n=96, seed=0):
+    if M <= n:
+        return None
+    rng = np.random.default_rng(seed)
+    pick = set(rng.choice(M, n - 4, replace=False).tolist()) | {0, 1, M - 2, M - 1}
+    return np.array(sorted(pick))
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_workload_parity(name):
+    """Full-size workloads: every code/scale byte compared for all rows, y and L
+    on a sample of rows (the oracle computes those rows one by one)."""
+    ck = synthetic.load(name)
+    layer = make_layer(ck)
+    x = dev_bf16(ck.x)
+    codes, scales, _ = layer.quantize_act(x, with_lowrank=False)
+    torch.cuda.synchronize()
+    c_ref, s_ref, _ = O.quantize_act(ck.x, ck.smooth_factor, ck.rotate_block)
+    np.testing.assert_array_equal(scales.cpu().numpy(), s_ref)
+    assert np.array_equal(codes.cpu().numpy(), c_ref)
+    rows = _sample_rows(ck.M)
+    check_quantizer(layer, ck, rows=rows)
+    check_forward(layer, ck, rows=rows)
+
+
+# ------------------------------------------------------------------ ragged shapes and edge cases
+
+@pytest.mark.parametrize("M,K,N,R,rot", [
+    (1, 256, 256, 32, 0),
+    (3, 48, 8, 16, 0),          # K < one chunk, N < one tile
+    (17, 272, 136, 48, 0),      # K % 128 != 0, N % 128 != 0, odd R
+    (129, 400, 200, 16, 0),     # M just over a tile, ragged everything
+    (200, 1024, 384, 128, 0),
+    (130, 384, 256, 32, 128),   # rotation, K = 3 rotation blocks
+    (64, 2048, 640, 64, 128),
+    (300, 4096, 128, 32, 0),    # split-K cluster reduction with ragged rows
+])
+def test_ragged_shapes(M, K, N, R, rot):
+    ck = synthetic.make_checkpoint(M, K, N, R, seed=M + K + N + R, rotate_block=rot, dense_weight=bool(rot),
+                                   wcscales="uniform", wtscale=0.75, name=f"ragged_{M}x{K}x{N}_r{R}_rot{rot}")
+    layer = make_layer(ck)
+    check_quantizer(layer, ck)
+    check_forward(layer, ck)
+
+
+def test_default_wcscales_wtscale_are_ones():
+    ck = synthetic.make_checkpoint(32, 256, 256, 32, seed=5)
+    layer = make_layer(ck, with_wc=False)
+    check_forward(layer, ck)
+
+
+def test_zero_weights_give_lowrank_branch_only():
+    ck = synthetic.make_checkpoint(40, 512, 256, 32, seed=6)
+    ck.qweight = np.zeros_like(ck.qweight)
+    layer = make_layer(ck)
+    y = check_forward(layer, ck)
+    xh = O.smooth_and_rotate(ck.x, ck.smooth_factor, 0)
+    lr = O.lowrank_down(xh, ck.proj_down) @ O.bf16_to_f32(ck.proj_up).astype(np.float64).T
+    assert_y_close(host_bf16_to_f64(y), lr, "lowrank only")
+
+
+def test_deterministic_and_batch_consistent():
+    ck = synthetic.make_checkpoint(300, 1024, 512, 32, seed=7)
+    layer = make_layer(ck)
+    x = dev_bf16(ck.x)
+    y1 = layer.forward(x).clone()
+    y2 = layer.forward(x).clone()
+    assert torch.equal(y1, y2)
+    y_one = layer.forward(x[5:6].contiguous())
+    assert torch.equal(y_one[0], y1[5])
+
+
+def test_zero_rows_is_noop():
+    ck = synthetic.make_checkpoint(4, 256, 256, 32, seed=8)
+    layer = make_layer(ck)
+    S.svdq_linear_forward(layer.handle, 0, 0, 0, 0)
+    assert S.svdq_workspace_bytes(layer.handle, 0) == 0
+
+
+def test_forward_host_matches_device_path():
+    ck = synthetic.make_checkpoint(64, 512, 384, 32, seed=9)
+    layer = make_layer(ck)
+    x = dev_bf16(ck.x)
+    y_dev_ref = layer.forward(x).clone()
+    xh = x.cpu().pin_memory()
+    yh = torch.empty((64, 384), dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty_like(x)
+    yd = torch.empty((64, 384), dtype=torch.bfloat16, device="cuda")
+    ws = layer.workspace(64)
+    S.svdq_linear_forward_host(layer.handle, xh.data_ptr(), 64, yh.data_ptr(), xd.data_ptr(), yd.data_ptr(),
+                               ws.data_ptr())
+    assert torch.equal(yh, y_dev_ref.cpu())
+
+
+def test_runtime_argument_errors():
+    ck = synthetic.make_checkpoint(4, 256, 256, 32, seed=10)
+    layer = make_layer(ck)
+    x = dev_bf16(ck.x)
+    y = torch.empty((4, 256), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(S.SvdqError) as e:
+        S.svdq_linear_forward(layer.handle, x.data_ptr(), 4, y.data_ptr(), 0)
+    assert e.value.status == 5
+    ws = layer.workspace(4)
+    with pytest.raises(S.SvdqError) as e:
+        S.svdq_linear_forward(layer.handle, x.data_ptr() + 2, 4, y.data_ptr(), ws.data_ptr())
+    assert e.value.status == 1
+    bad = synthetic.make_checkpoint(4, 256, 256, 32, seed=11)
+    bad.smooth_factor = bad.smooth_factor.copy()
+    bad.smooth_factor[3] = 0
+    with pytest.raises(S.SvdqError) as e:
+        make_layer(bad)
+    assert e.value.status == 1
