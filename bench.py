@@ -110,7 +110,7 @@ class ClockSampler:
                         self.reasons.add(k)
             except Exception:
                 pass
-            time.sleep(0.002)
+            time.sleep(0.0005)
 
     def __enter__(self):
         if self._nvml is not None:
@@ -126,7 +126,7 @@ class ClockSampler:
     def summary(self):
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples),
-                "source": "nvml, 2 ms period, during the timed region"}
+                "source": "nvml, 0.5 ms period, during the timed region"}
 
 
 def dist_setup():
@@ -272,8 +272,9 @@ def run_ours(args, world, rank, local):
     g_full = graph_of(args.steps, "both")
     g_quant = graph_of(args.steps, "quant")
     g_gemm = graph_of(args.steps, "gemm")
-    for g in (g_full, g_quant, g_gemm):        # graph warm-up replays
-        g.replay()
+    with torch.cuda.stream(stream):
+        for g in (g_full, g_quant, g_gemm):    # graph warm-up replays
+            g.replay()
     torch.cuda.synchronize()
     for lay, *_ in sets:
         if lay.device_status() != 0:
@@ -284,9 +285,10 @@ def run_ours(args, world, rank, local):
         e1 = torch.cuda.Event(enable_timing=True)
         barrier(world)
         torch.cuda.synchronize()
-        e0.record(stream)
-        g.replay()
-        e1.record(stream)
+        with torch.cuda.stream(stream):        # replay() launches on the current stream
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
         return e0.elapsed_time(e1) / 1e3
@@ -369,12 +371,12 @@ def run_ours(args, world, rank, local):
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rows = np.arange(min(M, args.ref_rows))
-        cpu_oracle_run(ck, rows[:16])
-        _, dt = cpu_oracle_run(ck, rows)
-        line["cpu_baseline"] = {"value": flops_per_step(len(rows), K, N, R) / dt / 1e12, "unit": "TFLOP/s",
-                                "cores": cpu_threads(), "kind": "oracle",
-                                "sample": f"{len(rows)} of {M} token rows of the workload, one run"}
+        cpu_oracle_run(ck, np.arange(16))
+        dts = [cpu_oracle_run(ck, None)[1] for _ in range(max(1, args.cpu_reps))]
+        dt = statistics.median(dts)
+        line["cpu_baseline"] = {"value": flops_per_step(M, K, N, R) / dt / 1e12, "unit": "TFLOP/s",
+                                "cores": cpu_threads(), "kind": "oracle", "seconds": sum(dts),
+                                "sample": f"the whole workload ({M} token rows), median of {len(dts)} runs"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     for lay, *_ in sets:
@@ -384,11 +386,14 @@ def run_ours(args, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=None)
-    ap.add_argument("--ref-rows", type=int, default=1024)
+    ap.add_argument("--ref-rows", type=int, default=256,
+                    help="token rows of the workload the reference arm (CPU oracle) runs per step")
+    ap.add_argument("--cpu-reps", type=int, default=3,
+                    help="full-workload oracle runs timed for cpu_baseline (median)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

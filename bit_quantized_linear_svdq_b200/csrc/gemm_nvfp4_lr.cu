@@ -8,17 +8,22 @@
 // bf16 rank correction of "Runtime support", fused here; shapes and scale
 // layout from "Checkpoint contract".)
 //
-// Per CTA: one 128 x 128 output tile.
-//   warp 0 lane 0   TMA producer: activation / weight code tiles (128 rows x
-//                   256 K as 128 swizzled bytes), their scale atoms (bulk
-//                   copies), and once per tile the L and proj_up tiles.
-//   warp 1          owns 512 TMEM columns; lane 0 copies each stage's scale
-//                   atoms to TMEM (tcgen05.cp) and issues the block-scaled
-//                   MMAs (M=128, N=128, K=64, UE4M3 per 16) into accumulator
-//                   columns [0,128); after the K loop it issues the bf16 MMAs
-//                   L . proj_up^T (K = R) into a second accumulator [128,256).
-//   warps 2-5       epilogue: TMEM -> registers, y = fma(alpha, acc, lr) ->
-//                   bf16 -> global.
+// Persistent kernel: one CTA per SM walks a static schedule of 128 x 128
+// output tiles (tile = blockIdx.x + i * gridDim.x, M-tile fastest).
+//   warp 0 lane 0   TMA producer: per K step (256 FP4 elements) the activation
+//                   and weight code tiles (128 rows x 128 swizzled bytes) and
+//                   their scale atoms (bulk copies) into a kStages ring; per
+//                   tile the L and proj_up tiles into a double buffer.
+//   warp 1          owns all 512 TMEM columns; lane 0 copies each stage's
+//                   scale atoms to TMEM (two tcgen05.cp .128x256b per operand;
+//                   a copy costs about the same whatever its size) and issues the
+//                   block-scaled MMAs (M=128, N=128, K=64, UE4M3 per 16) into
+//                   one of two accumulators; after the K loop it issues the
+//                   bf16 MMAs L . proj_up^T (K = R) into the rank-R accumulator.
+//   warps 2-5       epilogue of tile i (TMEM -> registers, y = fma(alpha, acc,
+//                   lr) -> bf16 -> global) while the tensor core runs tile i+1.
+// TMEM columns: accumulators [0,128) and [128,256), rank-R accumulator
+// [256,384), scale factors [384,448) (two buffers of A and B, 16 columns each).
 // Every wait is bounded; on expiry the CTA records an error, drains what it
 // started, frees TMEM and exits.
 #include <cuda_runtime.h>
@@ -31,17 +36,18 @@ namespace {
 
 constexpr int BM = 128, BN = 128;
 constexpr int kKTileBytes = 128;                 // 256 FP4 elements per row per stage
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kABytes = BM * kKTileBytes;        // 16 KB
 constexpr int kBBytes = BN * kKTileBytes;        // 16 KB
-constexpr int kSfaBytes = 4 * kSfAtomBytes;      // 4 K atoms x 128 rows
-constexpr int kSfbBytes = (BN / 128) * 4 * kSfAtomBytes;
-constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;   // 36 KB
+constexpr int kSfaBytes = 4 * kSfRepBytes;       // 4 replicated K atoms x 128 rows (8 KB)
+constexpr int kSfbBytes = (BN / 128) * 4 * kSfRepBytes;
+constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;   // 48 KB
 constexpr int kLrAtomBytesA = BM * 128;          // 64 bf16 of R per row
 constexpr int kLrAtomBytesB = BN * 128;
 constexpr int kThreads = 192;
+constexpr int kEpiWarps = 4;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColAcc = 0, kColLr = 128, kColSfa = 256, kColSfb = 288;   // SF: 2 buffers x 16
+constexpr uint32_t kColAcc = 0, kColLr = 256, kColSfa = 384, kColSfb = 416;   // SF: 2 buffers x 16
 
 struct GParams {
   const uint8_t* sfa;
@@ -50,37 +56,56 @@ struct GParams {
   __nv_bfloat16* y;
   unsigned* err;
   int M, N, R, k_tiles, ka_pad;
+  int m_tiles, n_tiles;
+  int lr_bufs;      // 2 when two L / proj_up tiles fit in shared memory, else 1
 };
+
+__device__ __forceinline__ void tile_coords(const GParams& p, int tile, int& mt, int& nt) {
+  mt = tile % p.m_tiles;
+  nt = tile / p.m_tiles;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nvfp4_lr_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                          const __grid_constant__ CUtensorMap tm_l, const __grid_constant__ CUtensorMap tm_pu,
                          const GParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // Round up to 1024 bytes by pointer arithmetic on the __shared__ array, so
+  // every access below stays a shared-memory access (an integer round trip
+  // would turn them into generic ones).
+  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int RA = (p.R + 63) / 64;              // 64-wide swizzled boxes covering R
+  const int lr_buf_bytes = RA * (kLrAtomBytesA + kLrAtomBytesB);
   uint8_t* stages = base;
-  uint8_t* LT = stages + kStages * kStageBytes;
-  uint8_t* PUT = LT + RA * kLrAtomBytesA;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(PUT + RA * kLrAtomBytesB);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + kStages;
-  uint64_t* lr_full = bars + 2 * kStages;
-  uint64_t* acc_full = bars + 2 * kStages + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 2);
+  uint8_t* LRB = stages + kStages * kStageBytes;          // lr_bufs x {L tile, proj_up tile}
+  uint64_t* bars = reinterpret_cast<uint64_t*>(LRB + p.lr_bufs * lr_buf_bytes);
+  uint64_t* full = bars;                        // [kStages] TMA landed
+  uint64_t* empty = full + kStages;             // [kStages] MMAs done reading the stage
+  uint64_t* lr_full = empty + kStages;          // [2] L / proj_up tile landed
+  uint64_t* lr_free = lr_full + 2;              // [2] rank-R MMAs done reading the L / proj_up tile
+  uint64_t* acc_full = lr_free + 2;             // [2] accumulator (and rank-R accumulator) ready
+  uint64_t* acc_free = acc_full + 2;            // [2] epilogue done reading accumulator
+  uint64_t* lracc_free = acc_free + 2;          // [1] epilogue done reading the rank-R accumulator
+  uint64_t* mma_done = lracc_free + 1;          // [1] every MMA of this CTA finished (teardown)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nt = blockIdx.x, mt = blockIdx.y;
-  const int n0 = nt * BN, m0 = mt * BM;
+  const int num_tiles = p.m_tiles * p.n_tiles;
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    mbar_init(smem_u32(lr_full), 1);
-    mbar_init(smem_u32(acc_full), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&lr_full[b]), 1);
+      mbar_init(smem_u32(&lr_free[b]), 1);
+      mbar_init(smem_u32(&acc_full[b]), 1);
+      mbar_init(smem_u32(&acc_free[b]), kEpiWarps);
+    }
+    mbar_init(smem_u32(lracc_free), kEpiWarps);
+    mbar_init(smem_u32(mma_done), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -93,34 +118,55 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  int issued = 0;
+  // Producer bookkeeping (for the drain after an abort).
+  int issued = 0, lr_issued = 0;
+
   if (warp == 0) {
     if (lane == 0) {
       prefetch_tmap(&tm_a);
       prefetch_tmap(&tm_b);
       prefetch_tmap(&tm_l);
       prefetch_tmap(&tm_pu);
-      const uint32_t lb = smem_u32(lr_full);
-      mbar_arrive_expect_tx(lb, (uint32_t)RA * (kLrAtomBytesA + kLrAtomBytesB));
-      for (int a = 0; a < RA; ++a) {
-        tma_load_2d(smem_u32(LT + a * kLrAtomBytesA), &tm_l, lb, 64 * a, m0);
-        tma_load_2d(smem_u32(PUT + a * kLrAtomBytesB), &tm_pu, lb, 64 * a, n0);
-      }
-      for (int kt = 0; kt < p.k_tiles; ++kt) {
-        const int s = kt % kStages;
-        if (kt >= kStages &&
-            !wait_bounded(smem_u32(&empty[s]), ((kt / kStages) - 1) & 1, abort_flag, p.err, kErrGemmTimeout))
-          break;
-        uint8_t* st = stages + s * kStageBytes;
-        const uint32_t fb = smem_u32(&full[s]);
-        mbar_arrive_expect_tx(fb, kStageBytes);
-        tma_load_2d(smem_u32(st), &tm_a, fb, kt * kKTileBytes, m0);
-        tma_load_2d(smem_u32(st + kABytes), &tm_b, fb, kt * kKTileBytes, n0);
-        bulk_load(smem_u32(st + kABytes + kBBytes),
-                  p.sfa + ((size_t)mt * p.ka_pad + (size_t)kt * 4) * kSfAtomBytes, kSfaBytes, fb);
-        bulk_load(smem_u32(st + kABytes + kBBytes + kSfaBytes),
-                  p.sfb + ((size_t)nt * p.ka_pad + (size_t)kt * 4) * kSfAtomBytes, kSfbBytes, fb);
-        issued = kt + 1;
+      int g = 0;   // k-stage counter across tiles
+      int it = 0;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+        int mt, nt;
+        tile_coords(p, tile, mt, nt);
+        const int m0 = mt * BM, n0 = nt * BN;
+        // L / proj_up tile of this output tile.
+        {
+          const int lb = p.lr_bufs == 2 ? (it & 1) : 0;
+          const int use = p.lr_bufs == 2 ? (it >> 1) : it;
+          if (use >= 1 && !wait_bounded(smem_u32(&lr_free[lb]), (use - 1) & 1, abort_flag, p.err, kErrGemmTimeout))
+            break;
+          uint8_t* lt = LRB + lb * lr_buf_bytes;
+          const uint32_t fb = smem_u32(&lr_full[lb]);
+          mbar_arrive_expect_tx(fb, (uint32_t)lr_buf_bytes);
+          for (int a = 0; a < RA; ++a) {
+            tma_load_2d(smem_u32(lt + a * kLrAtomBytesA), &tm_l, fb, 64 * a, m0);
+            tma_load_2d(smem_u32(lt + RA * kLrAtomBytesA + a * kLrAtomBytesB), &tm_pu, fb, 64 * a, n0);
+          }
+          lr_issued = it + 1;
+        }
+        bool stop = false;
+        for (int kt = 0; kt < p.k_tiles; ++kt, ++g) {
+          const int s = g % kStages, n = g / kStages;
+          if (n >= 1 && !wait_bounded(smem_u32(&empty[s]), (n - 1) & 1, abort_flag, p.err, kErrGemmTimeout)) {
+            stop = true;
+            break;
+          }
+          uint8_t* st = stages + s * kStageBytes;
+          const uint32_t fb = smem_u32(&full[s]);
+          mbar_arrive_expect_tx(fb, kStageBytes);
+          tma_load_2d(smem_u32(st), &tm_a, fb, kt * kKTileBytes, m0);
+          tma_load_2d(smem_u32(st + kABytes), &tm_b, fb, kt * kKTileBytes, n0);
+          bulk_load(smem_u32(st + kABytes + kBBytes),
+                    p.sfa + ((size_t)mt * p.ka_pad + (size_t)kt * 4) * kSfRepBytes, kSfaBytes, fb);
+          bulk_load(smem_u32(st + kABytes + kBBytes + kSfaBytes),
+                    p.sfb + ((size_t)nt * p.ka_pad + (size_t)kt * 4) * kSfRepBytes, kSfbBytes, fb);
+          issued = g + 1;
+        }
+        if (stop) break;
       }
     }
     __syncwarp();
@@ -128,80 +174,120 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_main = idesc_nvfp4(BM, BN);
       const uint32_t idesc_lr = idesc_bf16_f32(BM, BN);
+      int g = 0;
+      int it = 0;
       bool ok = true;
-      for (int kt = 0; kt < p.k_tiles; ++kt) {
-        const int s = kt % kStages;
-        if (!wait_bounded(smem_u32(&full[s]), (kt / kStages) & 1, abort_flag, p.err, kErrGemmTimeout)) {
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+        const int ab = it & 1;
+        const uint32_t acc = tmem + kColAcc + (uint32_t)ab * BN;
+        if (it >= 2 && !wait_bounded(smem_u32(&acc_free[ab]), ((it >> 1) - 1) & 1, abort_flag, p.err, kErrGemmTimeout)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
-        const uint32_t st = smem_u32(stages + s * kStageBytes);
-        const uint32_t sfa_col = kColSfa + (uint32_t)(kt & 1) * 16u;
-        const uint32_t sfb_col = kColSfb + (uint32_t)(kt & 1) * 16u;
+        for (int kt = 0; kt < p.k_tiles; ++kt, ++g) {
+          const int s = g % kStages, n = g / kStages;
+          if (!wait_bounded(smem_u32(&full[s]), n & 1, abort_flag, p.err, kErrGemmTimeout)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t st = smem_u32(stages + s * kStageBytes);
+          const uint32_t sfa_col = kColSfa + (uint32_t)(g & 1) * 16u;
+          const uint32_t sfb_col = kColSfb + (uint32_t)(g & 1) * 16u;
+          // Scale factors: one 128 x 256-bit copy per operand and pair of K atoms
+          // (replicated atoms kb and kb+1 are 2 KB apart; columns 4 kb .. 4 kb + 7).
 #pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-          tmem_cp_32x128b_x4(tmem + sfa_col + kb * 4, sdesc_sf_atom(st + kABytes + kBBytes + kb * kSfAtomBytes));
-          tmem_cp_32x128b_x4(tmem + sfb_col + kb * 4,
-                             sdesc_sf_atom(st + kABytes + kBBytes + kSfaBytes + kb * kSfAtomBytes));
-        }
+          for (int kb = 0; kb < 4; kb += 2) {
+            tmem_cp_128x256b(tmem + sfa_col + kb * 4, sdesc_rows32b(st + kABytes + kBBytes + kb * kSfRepBytes, kSfRepBytes));
+            tmem_cp_128x256b(tmem + sfb_col + kb * 4,
+                             sdesc_rows32b(st + kABytes + kBBytes + kSfaBytes + kb * kSfRepBytes, kSfRepBytes));
+          }
 #pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-          mma_nvfp4(tmem + kColAcc, sdesc_kmajor_sw128(st + kb * 32), sdesc_kmajor_sw128(st + kABytes + kb * 32),
-                    idesc_main, tmem + sfa_col + kb * 4, tmem + sfb_col + kb * 4, (kt | kb) != 0);
+          for (int kb = 0; kb < 4; ++kb) {
+            mma_nvfp4(acc, sdesc_kmajor_sw128(st + kb * 32), sdesc_kmajor_sw128(st + kABytes + kb * 32), idesc_main,
+                      tmem + sfa_col + kb * 4, tmem + sfb_col + kb * 4, (kt | kb) != 0);
+          }
+          tc_commit(smem_u32(&empty[s]));
         }
-        tc_commit(smem_u32(&empty[s]));
-      }
-      if (ok && wait_bounded(smem_u32(lr_full), 0, abort_flag, p.err, kErrGemmTimeout)) {
+        if (!ok) break;
+        // rank-R correction into its own accumulator
+        const int lb = p.lr_bufs == 2 ? (it & 1) : 0;
+        const int use = p.lr_bufs == 2 ? (it >> 1) : it;
+        if (!wait_bounded(smem_u32(&lr_full[lb]), use & 1, abort_flag, p.err, kErrGemmTimeout) ||
+            (it >= 1 && !wait_bounded(smem_u32(lracc_free), (it - 1) & 1, abort_flag, p.err, kErrGemmTimeout))) {
+          ok = false;
+          break;
+        }
         tc_fence_after_sync();
-        const uint32_t la = smem_u32(LT), pa = smem_u32(PUT);
+        const uint32_t la = smem_u32(LRB + lb * lr_buf_bytes);
+        const uint32_t pa = la + RA * kLrAtomBytesA;
         for (int kk = 0; kk < p.R / 16; ++kk) {
           mma_bf16(tmem + kColLr, sdesc_kmajor_sw128(la + (kk >> 2) * kLrAtomBytesA + (kk & 3) * 32),
                    sdesc_kmajor_sw128(pa + (kk >> 2) * kLrAtomBytesB + (kk & 3) * 32), idesc_lr, kk != 0);
         }
+        tc_commit(smem_u32(&lr_free[lb]));
+        tc_commit(smem_u32(&acc_full[ab]));
       }
-      tc_commit(smem_u32(acc_full));
     }
     __syncwarp();
   } else {
     // Epilogue: warps 2..5 cover TMEM lane quadrants 2, 3, 0, 1.
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    const int m = m0 + row;
-    const bool ok = wait_bounded(smem_u32(acc_full), 0, abort_flag, p.err, kErrGemmTimeout);
-    tc_fence_after_sync();
-    if (ok && !*abort_flag) {
-      const bool vec_ok = (p.N & 7) == 0;
+    const bool vec_ok = (p.N & 7) == 0;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      int mt, nt;
+      tile_coords(p, tile, mt, nt);
+      const int m = mt * BM + row, n0 = nt * BN;
+      const int ab = it & 1;
+      if (!wait_bounded(smem_u32(&acc_full[ab]), (it >> 1) & 1, abort_flag, p.err, kErrGemmTimeout)) break;
+      tc_fence_after_sync();
+      const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
       for (int j = 0; j < BN / 32; ++j) {
         uint32_t acc[32], lr[32];
-        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + kColAcc + j * 32, acc);
-        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + kColLr + j * 32, lr);
+        tmem_ld32(lane_base + kColAcc + (uint32_t)ab * BN + j * 32, acc);
+        tmem_ld32(lane_base + kColLr + j * 32, lr);
         tmem_ld_wait();
+        if (j == BN / 32 - 1) {
+          // Both accumulators of this tile are in registers: release them.
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(smem_u32(&acc_free[ab]));
+            mbar_arrive(smem_u32(lracc_free));
+          }
+        }
         const int n = n0 + j * 32;
         if (m < p.M && n < p.N) {
           const float4* al = reinterpret_cast<const float4*>(p.alpha + n);
-          uint32_t packed[16];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const float4 a4 = __ldg(al + c);
-            const float y0 = fmaf(a4.x, __uint_as_float(acc[4 * c + 0]), __uint_as_float(lr[4 * c + 0]));
-            const float y1 = fmaf(a4.y, __uint_as_float(acc[4 * c + 1]), __uint_as_float(lr[4 * c + 1]));
-            const float y2 = fmaf(a4.z, __uint_as_float(acc[4 * c + 2]), __uint_as_float(lr[4 * c + 2]));
-            const float y3 = fmaf(a4.w, __uint_as_float(acc[4 * c + 3]), __uint_as_float(lr[4 * c + 3]));
-            packed[2 * c] = pack_bf16x2(y0, y1);
-            packed[2 * c + 1] = pack_bf16x2(y2, y3);
-          }
           __nv_bfloat16* dst = p.y + (size_t)m * p.N + n;
           if (vec_ok && n + 32 <= p.N) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-              d4[c] = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+            for (int c = 0; c < 4; ++c) {
+              const float4 a0 = __ldg(al + 2 * c), a1 = __ldg(al + 2 * c + 1);
+              const int b = 8 * c;
+              uint4 o;
+              o.x = pack_bf16x2(fmaf(a0.x, __uint_as_float(acc[b + 0]), __uint_as_float(lr[b + 0])),
+                                fmaf(a0.y, __uint_as_float(acc[b + 1]), __uint_as_float(lr[b + 1])));
+              o.y = pack_bf16x2(fmaf(a0.z, __uint_as_float(acc[b + 2]), __uint_as_float(lr[b + 2])),
+                                fmaf(a0.w, __uint_as_float(acc[b + 3]), __uint_as_float(lr[b + 3])));
+              o.z = pack_bf16x2(fmaf(a1.x, __uint_as_float(acc[b + 4]), __uint_as_float(lr[b + 4])),
+                                fmaf(a1.y, __uint_as_float(acc[b + 5]), __uint_as_float(lr[b + 5])));
+              o.w = pack_bf16x2(fmaf(a1.z, __uint_as_float(acc[b + 6]), __uint_as_float(lr[b + 6])),
+                                fmaf(a1.w, __uint_as_float(acc[b + 7]), __uint_as_float(lr[b + 7])));
+              reinterpret_cast<uint4*>(dst)[c] = o;
+            }
           } else {
-            const uint16_t* h = reinterpret_cast<const uint16_t*>(packed);
-            uint16_t* d = reinterpret_cast<uint16_t*>(dst);
-            for (int c = 0; c < 32 && n + c < p.N; ++c) d[c] = h[c];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              if (n + c < p.N) {
+                const float v = fmaf(p.alpha[n + c], __uint_as_float(acc[c]), __uint_as_float(lr[c]));
+                dst[c] = __float2bfloat16_rn(v);
+              }
+            }
           }
         }
       }
@@ -214,9 +300,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int last = s + ((issued - 1 - s) / kStages) * kStages;
       wait_for(smem_u32(&full[s]), (last / kStages) & 1, 100000000ull);
     }
-    wait_for(smem_u32(lr_full), 0, 100000000ull);
+    for (int b = 0; b < p.lr_bufs && b < lr_issued; ++b) {
+      const int last_it = b + ((lr_issued - 1 - b) / p.lr_bufs) * p.lr_bufs;
+      const int use = p.lr_bufs == 2 ? (last_it >> 1) : last_it;
+      wait_for(smem_u32(&lr_full[b]), use & 1, 100000000ull);
+    }
   }
-  if (warp == 1 && lane == 0) wait_for(smem_u32(acc_full), 0, kWaitTimeoutNs);
+  if (warp == 1 && lane == 0) {
+    // No MMA may still be running when the tensor memory is released.
+    tc_commit(smem_u32(mma_done));
+    wait_for(smem_u32(mma_done), 0, kWaitTimeoutNs);
+  }
   tc_fence_before_sync();
   __syncthreads();
   if (warp == 1) {
@@ -230,9 +324,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 cudaError_t launch_gemm_nvfp4_lr(const GemmLaunch& L, cudaStream_t stream) {
   if (L.M <= 0) return cudaSuccess;
   const int RA = (L.R + 63) / 64;
-  const size_t smem = 1024 + (size_t)kStages * kStageBytes + (size_t)RA * (kLrAtomBytesA + kLrAtomBytesB) + 256;
+  const int lr_buf_bytes = RA * (kLrAtomBytesA + kLrAtomBytesB);
+  const size_t fixed = 1024 + (size_t)kStages * kStageBytes + 256;
+  const int lr_bufs = (fixed + 2 * (size_t)lr_buf_bytes <= 227 * 1024) ? 2 : 1;
+  const size_t smem = fixed + (size_t)lr_bufs * lr_buf_bytes;
   cudaError_t e = ensure_smem_limit(gemm_nvfp4_lr_kernel, smem);
   if (e != cudaSuccess) return e;
+  static int num_sms = 0;
+  if (num_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (num_sms <= 0) num_sms = 148;
+  }
   GParams p;
   p.sfa = L.sfa;
   p.sfb = L.sfb;
@@ -244,7 +348,11 @@ cudaError_t launch_gemm_nvfp4_lr(const GemmLaunch& L, cudaStream_t stream) {
   p.R = L.R;
   p.k_tiles = L.k_tiles;
   p.ka_pad = L.ka_pad;
-  dim3 grid((unsigned)((L.N + BN - 1) / BN), (unsigned)((L.M + BM - 1) / BM), 1);
+  p.m_tiles = (L.M + BM - 1) / BM;
+  p.n_tiles = (L.N + BN - 1) / BN;
+  p.lr_bufs = lr_bufs;
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int grid = tiles < num_sms ? tiles : num_sms;
   gemm_nvfp4_lr_kernel<<<grid, kThreads, smem, stream>>>(L.tm_a, L.tm_b, L.tm_l, L.tm_pu, p);
   return cudaGetLastError();
 }

@@ -163,6 +163,12 @@ __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdes
                : "memory");
 }
 
+// Copy a 128-row x 256-bit shared-memory matrix into TMEM lanes 0-127,
+// columns [taddr, taddr+8): row r -> lane r.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -206,6 +212,14 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
 // swizzle, 8-row core matrices 128 bytes apart) as the source of tcgen05.cp.
 __device__ __forceinline__ uint64_t sdesc_sf_atom(uint32_t saddr) {
   return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(128u >> 4) << 32) | (1ull << 46);
+}
+
+// Descriptor of a 128-row x 32-byte shared-memory matrix without swizzle:
+// bytes 0-15 of row r at saddr + 16 r, bytes 16-31 at saddr + lbo + 16 r
+// (8-row core matrices 128 bytes apart), the source of tcgen05.cp .128x256b.
+__device__ __forceinline__ uint64_t sdesc_rows32b(uint32_t saddr, uint32_t lbo) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)(128u >> 4) << 32) | (1ull << 46);
 }
 
 // Instruction descriptor: kind::f16 with bf16 A/B, fp32 D, both K-major.

@@ -14,19 +14,32 @@
 // Work decomposition.  A CTA owns 128 token rows and a contiguous slice of
 // K; the K slices of one row tile form a thread-block cluster that reduces
 // its partial L in distributed shared memory (fixed order, deterministic).
-// Inside a CTA:
-//   warp 4 lane 0   TMA producer: x chunk (128 rows x 128 K, two 128B-swizzled
-//                   boxes), proj_down^T chunk (R x 128) and {smooth, 1/smooth}
-//                   into a STAGES-deep ring; also owns the TMEM allocation.
-//   warps 0-3       one thread per row: smooth (+ rotate), quantize, write
-//                   codes/scales to global, and write bf16(x_hat) back in place
-//                   over x in shared memory -- which is exactly the 128B-swizzled
-//                   K-major layout the tensor core reads as the A operand.
-//   warp 5 lane 0   issues tcgen05.mma (M=128, N=R, K=16, bf16 -> fp32 TMEM)
+// Inside a CTA (320 threads; two CTAs per SM without rotation):
+//   warp 8 lane 0   TMA producer: x chunk (128 rows x 128 K, two 128B-swizzled
+//                   boxes), proj_down^T chunk (R x 128) and the smooth factors
+//                   into a 2-deep ring; warp 8 also owns the TMEM allocation.
+//   warps 0-7       two threads per row, 64 K elements each: smooth (+ rotate),
+//                   quantize, write codes/scales to global, and write bf16(x_hat)
+//                   back in place over x in shared memory -- exactly the
+//                   128B-swizzled K-major layout the tensor core reads as A.
+//   warp 9 lane 0   issues tcgen05.mma (M=128, N=R, K=16, bf16 -> fp32 TMEM)
 //                   for L on each finished chunk, releasing the stage when done.
+//
+// Exact fp32 division without the divide unit: with y = RN(1/b),
+//   q0 = RN(a*y), r = RN(a - b*q0) (fused), q1 = RN(q0 + r*y) (fused)
+// is the correctly rounded a/b (Markstein's iteration; checked exhaustively
+// for every significand pair that occurs here: bf16/bf16 for the smoothing,
+// fp32/e4m3 and fp32/6 for the scale and codes).  The reciprocals come from
+// create time (1/smooth) and a per-CTA table over the 127 e4m3 scales.  Two
+// lanes run per instruction (fma.rn.f32x2).  Blocks whose values overflow or
+// hold NaN take an IEEE-division slow path, so results equal the divide
+// unit's in every case.
+//
 // Every wait is bounded (kWaitTimeoutNs); on expiry the CTA records an error,
 // drains what it started, frees TMEM and exits.
 #include <cuda_runtime.h>
+
+#include <cstdlib>
 
 #include "kcommon.cuh"
 #include "svdq_kernels.h"
@@ -34,15 +47,18 @@
 namespace svdq {
 namespace {
 
-constexpr int kChunk = 128;           // K elements per pipeline stage
-constexpr int kRows = 128;            // token rows per CTA (TMEM lanes)
+constexpr int kChunk = 128;                        // K elements per pipeline stage
+constexpr int kRows = 128;                         // token rows per CTA (TMEM lanes)
+constexpr int kStages = 2;
 constexpr int kXStageBytes = kRows * kChunk * 2;   // 32 KB: two 64-wide swizzled boxes
 constexpr int kXBoxBytes = kXStageBytes / 2;       // 16 KB
-constexpr int kLamStageBytes = kChunk * 8;         // float2 per channel
-constexpr int kThreads = 192;
+constexpr int kLamStageBytes = kChunk * 8;         // float4 {-s0,-s1,1/s0,1/s1} per channel pair
+constexpr int kComputeThreads = 256;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = 320;
 
 struct QParams {
-  const float2* lam2;
+  const float4* lam4;
   uint8_t* codes;
   uint8_t* scales;
   __nv_bfloat16* lowrank;
@@ -52,36 +68,75 @@ struct QParams {
   int chunks_per_cta, n_chunks, ksplit;
 };
 
-// Quantize one 16-element block: returns the scale byte, writes 16 codes as two words.
-__device__ __forceinline__ uint32_t quant_block16(const float* v, uint32_t& w0, uint32_t& w1) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-  const uint32_t sb = cvt_e4m3(__fdiv_rn(amax, 6.0f));
-  const float s = e4m3_to_f32(sb);
-  if (s > 0.0f) {
-    float q[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(v[i], s);
-    w0 = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
-    w1 = cvt_e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
-  } else {
-    w0 = 0u;
-    w1 = 0u;
-  }
-  return sb;
+// ---------------------------------------------------------------- packed fp32 helpers
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float lo2(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi2(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
 }
 
-__device__ __forceinline__ void unpack8(const uint4& p, float* v) {
-  v[0] = bf16lo_to_f32(p.x); v[1] = bf16hi_to_f32(p.x);
-  v[2] = bf16lo_to_f32(p.y); v[3] = bf16hi_to_f32(p.y);
-  v[4] = bf16lo_to_f32(p.z); v[5] = bf16hi_to_f32(p.z);
-  v[6] = bf16lo_to_f32(p.w); v[7] = bf16hi_to_f32(p.w);
+// Correctly rounded a / B for two lanes, given nb = -B and y = RN(1 / B).
+// Zero results may carry the wrong sign (q0 + r*y with r = +0).
+__device__ __forceinline__ uint64_t div_mk2(uint64_t a, uint64_t nb, uint64_t y) {
+  const uint64_t q0 = mul2(a, y);
+  const uint64_t r = fma2(q0, nb, a);
+  return fma2(r, y, q0);
 }
 
-__device__ __forceinline__ uint4 pack8(const float* v) {
-  return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                    pack_bf16x2(v[6], v[7]));
+// As div_mk2, but the result keeps the sign of a*y, so a signed zero divides
+// to a correctly signed zero for any divisor.
+__device__ __forceinline__ uint64_t div_rn2(uint64_t a, uint64_t nb, uint64_t y) {
+  const uint64_t q0 = mul2(a, y);
+  const uint64_t r = fma2(q0, nb, a);
+  const uint64_t q1 = fma2(r, y, q0);
+  return (q1 & 0x7FFFFFFF7FFFFFFFull) | (q0 & 0x8000000080000000ull);
+}
+
+// With a negative divisor B = -b (b > 0), div_mk2 returns correctly signed
+// zeros as well: a = +-0 gives q0 = -+0, r = +0 and q1 = -+0 = a / B.  The
+// "negated" layout divides x by -smooth (giving -x_hat exactly) and -x_hat by
+// -scale (giving x_hat / scale), so no sign fix-up is needed when every smooth
+// factor is positive.
+
+// max(acc, |v|) that propagates NaN (the scale of a block holding a NaN is NaN).
+__device__ __forceinline__ float amax_nan(float acc, float v) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(acc), "f"(fabsf(v)));
+  return r;
+}
+
+__device__ __forceinline__ float amax8(const uint64_t (&v)[8]) {
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = amax_nan(amax_nan(a, lo2(v[i])), hi2(v[i]));
+  return a;
+}
+
+// bf16 word (two channels) -> packed fp32 pair
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
+  return pk2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
 // Byte offset, inside one stage's x tile, of the 16-byte group `c` (8 bf16,
@@ -91,89 +146,287 @@ __device__ __forceinline__ uint32_t xoff(int row, int c) {
   return (uint32_t)((c >> 3) * kXBoxBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4));
 }
 
-// Global writes of one quantized 16-element block.
+struct Tables {
+  // e4m3 code -> {-B, RN(1/B)} for the scale division: B = s (sign-fixed
+  // layout) or B = -s (negated layout).  Entry 0 is unused.
+  float2 srec[128];
+};
+
+// Quantize one 16-element block held as 8 packed pairs of finite values:
+// returns the scale byte and the 16 codes (w0: elements 0-7, w1: 8-15).
+template <bool NEG>
+__device__ __forceinline__ uint32_t quant_block(const uint64_t (&v)[8], float amax, const float2* srec, float y6,
+                                                uint32_t& w0, uint32_t& w1) {
+  // amax / 6, correctly rounded (Markstein with y6 = RN(1/6)).
+  const float q0 = amax * y6;
+  const float q1 = fmaf(fmaf(q0, -6.0f, amax), y6, q0);
+  const uint32_t sb = cvt_e4m3(q1);
+  w0 = w1 = 0u;
+  if (sb != 0u) {
+    const float2 sr = srec[sb];
+    const uint64_t ns = pk2(sr.x, sr.x), ys = pk2(sr.y, sr.y);
+    uint64_t q[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q[i] = NEG ? div_mk2(v[i], ns, ys) : div_rn2(v[i], ns, ys);
+    w0 = cvt_e2m1x8(lo2(q[0]), hi2(q[0]), lo2(q[1]), hi2(q[1]), lo2(q[2]), hi2(q[2]), lo2(q[3]), hi2(q[3]));
+    w1 = cvt_e2m1x8(lo2(q[4]), hi2(q[4]), lo2(q[5]), hi2(q[5]), lo2(q[6]), hi2(q[6]), lo2(q[7]), hi2(q[7]));
+  }
+  return sb;
+}
+
+// IEEE-division path for blocks holding +-inf or NaN.
+__device__ __forceinline__ uint32_t quant_block_slow(const uint64_t (&v)[8], uint32_t& w0, uint32_t& w1) {
+  float f[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    f[2 * i] = lo2(v[i]);
+    f[2 * i + 1] = hi2(v[i]);
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = amax_nan(amax, f[i]);
+  const uint32_t sb = cvt_e4m3(__fdiv_rn(amax, 6.0f));
+  const float s = e4m3_to_f32(sb);
+  w0 = w1 = 0u;
+  if (s > 0.0f) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) f[i] = __fdiv_rn(f[i], s);
+    w0 = cvt_e2m1x8(f[0], f[1], f[2], f[3], f[4], f[5], f[6], f[7]);
+    w1 = cvt_e2m1x8(f[8], f[9], f[10], f[11], f[12], f[13], f[14], f[15]);
+  }
+  return sb;
+}
+
+__device__ __forceinline__ uint32_t quantize_any(const uint64_t (&v)[8], const float2* srec, float y6, uint32_t& w0,
+                                                 uint32_t& w1) {
+  const float amax = amax8(v);
+  return (amax < 3.0e38f) ? quant_block<false>(v, amax, srec, y6, w0, w1) : quant_block_slow(v, w0, w1);
+}
+
+__device__ __forceinline__ void write_back_bf16(uint8_t* xs, int row, int c0, const uint64_t (&v)[8]) {
+  uint4 o0, o1;
+  o0.x = pack_bf16x2(lo2(v[0]), hi2(v[0])); o0.y = pack_bf16x2(lo2(v[1]), hi2(v[1]));
+  o0.z = pack_bf16x2(lo2(v[2]), hi2(v[2])); o0.w = pack_bf16x2(lo2(v[3]), hi2(v[3]));
+  o1.x = pack_bf16x2(lo2(v[4]), hi2(v[4])); o1.y = pack_bf16x2(lo2(v[5]), hi2(v[5]));
+  o1.z = pack_bf16x2(lo2(v[6]), hi2(v[6])); o1.w = pack_bf16x2(lo2(v[7]), hi2(v[7]));
+  *reinterpret_cast<uint4*>(xs + xoff(row, c0)) = o0;
+  *reinterpret_cast<uint4*>(xs + xoff(row, c0 + 1)) = o1;
+}
+
 template <bool TILED>
-__device__ __forceinline__ void store_block(const QParams& p, int m, int row_in_tile, int k,
-                                            uint32_t w0, uint32_t w1, uint32_t sb) {
-  if (k >= p.k_limit) return;
-  *reinterpret_cast<uint2*>(p.codes + (size_t)m * p.codes_pitch + (k >> 1)) = make_uint2(w0, w1);
-  if (TILED) {
-    const int ka = k >> 6, j = (k >> 4) & 3;
-    p.scales[((size_t)(m >> 7) * p.ka_pad + ka) * kSfAtomBytes + sf_atom_offset(row_in_tile, j)] =
-        (uint8_t)sb;
+__device__ __forceinline__ void store_codes(const QParams& p, int m, int k, const uint32_t (&w)[8]) {
+  // 64 K elements = 32 code bytes of one row, starting at element k.
+  uint8_t* dst = p.codes + (size_t)m * p.codes_pitch + (k >> 1);
+  if (k + 64 <= p.k_limit) {
+    if (TILED) {   // workspace rows are 16-byte aligned
+      reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    } else {       // caller rows are 8-byte aligned (K % 16 == 0)
+      uint2* d = reinterpret_cast<uint2*>(dst);
+      d[0] = make_uint2(w[0], w[1]);
+      d[1] = make_uint2(w[2], w[3]);
+      d[2] = make_uint2(w[4], w[5]);
+      d[3] = make_uint2(w[6], w[7]);
+    }
   } else {
-    p.scales[(size_t)m * p.scales_pitch + (k >> 4)] = (uint8_t)sb;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (k + 16 * j < p.k_limit) reinterpret_cast<uint2*>(dst)[j] = make_uint2(w[2 * j], w[2 * j + 1]);
   }
 }
 
-template <bool ROT, bool TILED>
-__device__ __forceinline__ void process_chunk(const QParams& p, uint8_t* xs, const float2* lam,
-                                              int row, int m, int kc) {
-  const bool valid = m < p.M;
-  if (ROT) {
-    // The whole 128-element rotation block of this row lives in registers.
-    float v[128];
+template <bool TILED>
+__device__ __forceinline__ void store_scales(const QParams& p, int m, int row, int k, uint32_t sbytes) {
+  // four scale bytes (16-element blocks k/16 .. k/16+3), byte j for block j
+  if (TILED) {
+    uint8_t* atom = p.scales + ((size_t)(m >> 7) * p.ka_pad + (k >> 6)) * kSfRepBytes + sf_atom_offset(row, 0);
 #pragma unroll
-    for (int c = 0; c < 16; ++c) unpack8(*reinterpret_cast<const uint4*>(xs + xoff(row, c)), v + 8 * c);
+    for (int r = 0; r < 4; ++r) *reinterpret_cast<uint32_t*>(atom + r * kSfAtomBytes) = sbytes;
+  } else {
+    uint8_t* dst = p.scales + (size_t)m * p.scales_pitch + (k >> 4);
+    if (k + 64 <= p.k_limit && ((reinterpret_cast<uintptr_t>(dst) & 3u) == 0)) {
+      *reinterpret_cast<uint32_t*>(dst) = sbytes;
+    } else {
 #pragma unroll
-    for (int i = 0; i < 128; ++i) v[i] = __fdiv_rn(v[i], lam[i].x);
-    // Walsh-Hadamard butterfly, stages h = 1, 2, ..., 64, fp32 adds.
+      for (int j = 0; j < 4; ++j)
+        if (k + 16 * j < p.k_limit) dst[j] = (uint8_t)(sbytes >> (8 * j));
+    }
+  }
+}
+
+// Rotated path, one thread: the 64 consecutive K elements (half `q` of the
+// chunk, one 128-element rotation block per row) of row `row`.  Codes and
+// scale bytes are returned in registers and stored after the chunk is handed
+// to the tensor core.
+__device__ __forceinline__ void rotate_half(uint8_t* xs, const float4* lam4, const float2* srec, float y6, int row,
+                                            int q, uint32_t (&cw)[8], uint32_t& sbytes) {
+  const float4* lam = lam4 + 32 * q;          // the 32 channel pairs of this half
+  sbytes = 0;
+  // The row's 128-element rotation block is split over lanes 2r (first 64)
+  // and 2r+1 (last 64) of one warp.  Element e of this half is lane (e & 1)
+  // of v[e >> 1].
+  uint64_t v[32];
+  float big = 0.0f;
 #pragma unroll
-    for (int h = 1; h < 128; h <<= 1) {
+  for (int c = 0; c < 8; ++c) {
+    const uint4 pw = *reinterpret_cast<const uint4*>(xs + xoff(row, 8 * q + c));
+    const uint32_t xin[4] = {pw.x, pw.y, pw.z, pw.w};
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        if ((i & h) == 0) {
-          const float a = v[i], b = v[i + h];
-          v[i] = __fadd_rn(a, b);
-          v[i + h] = __fsub_rn(a, b);
-        }
+    for (int i = 0; i < 4; ++i) {
+      const float4 l = lam[4 * c + i];
+      v[4 * c + i] = div_rn2(bf16x2_to_f2(xin[i]), pk2(l.x, l.y), pk2(l.z, l.w));
+      big = amax_nan(amax_nan(big, lo2(v[4 * c + i])), hi2(v[4 * c + i]));
+    }
+  }
+  if (!(big < 3.0e38f)) {            // overflow / NaN (rare): redo with the divide unit
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 pw = *reinterpret_cast<const uint4*>(xs + xoff(row, 8 * q + c));
+      const uint32_t xin[4] = {pw.x, pw.y, pw.z, pw.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 l = lam[4 * c + i];
+        v[4 * c + i] = pk2(__fdiv_rn(__uint_as_float(xin[i] << 16), -l.x),
+                           __fdiv_rn(__uint_as_float(xin[i] & 0xFFFF0000u), -l.y));
       }
     }
-    const float cnorm = 0.0883883461356163f;   // fp32(1/sqrt(128)) = 0x3DB504F3
+  }
+  // Butterfly stage h = 1: the pair (2i, 2i+1) is the two lanes of v[i];
+  // regroup two words so each packed op yields two results.
 #pragma unroll
-    for (int i = 0; i < 128; ++i) v[i] = __fmul_rn(v[i], cnorm);
+  for (int j = 0; j < 16; ++j) {
+    const uint64_t a = pk2(lo2(v[2 * j]), lo2(v[2 * j + 1]));
+    const uint64_t b = pk2(hi2(v[2 * j]), hi2(v[2 * j + 1]));
+    const uint64_t sm = add2(a, b), df = sub2(a, b);
+    v[2 * j] = pk2(lo2(sm), lo2(df));
+    v[2 * j + 1] = pk2(hi2(sm), hi2(df));
+  }
+  // Stages h = 2, 4, 8, 16, 32: pairs of packed words (i, i + h/2).
 #pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      uint32_t w0, w1;
-      const uint32_t sb = quant_block16(v + 16 * b, w0, w1);
-      if (valid) store_block<TILED>(p, m, row, kc + 16 * b, w0, w1, sb);
-      *reinterpret_cast<uint4*>(xs + xoff(row, 2 * b)) = pack8(v + 16 * b);
-      *reinterpret_cast<uint4*>(xs + xoff(row, 2 * b + 1)) = pack8(v + 16 * b + 8);
+  for (int st = 0; st < 5; ++st) {
+    const int hp = 1 << st;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if ((i & hp) == 0) {
+        const uint64_t a = v[i], b = v[i + hp];
+        v[i] = add2(a, b);
+        v[i + hp] = sub2(a, b);
+      }
     }
-  } else {
-#pragma unroll 2
-    for (int b = 0; b < 8; ++b) {
-      float v[16];
-      unpack8(*reinterpret_cast<const uint4*>(xs + xoff(row, 2 * b)), v);
-      unpack8(*reinterpret_cast<const uint4*>(xs + xoff(row, 2 * b + 1)), v + 8);
+  }
+  // Stage h = 64 across the lane pair: lower half a + b, upper half a - b,
+  // each one fused op (+-mine + other) with a single rounding.
+  {
+    const float sg = q ? -1.0f : 1.0f;
+    const uint64_t sg2 = pk2(sg, sg);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = __fdiv_rn(v[i], lam[16 * b + i].x);
-      uint32_t w0, w1;
-      const uint32_t sb = quant_block16(v, w0, w1);
-      if (valid) store_block<TILED>(p, m, row, kc + 16 * b, w0, w1, sb);
-      *reinterpret_cast<uint4*>(xs + xoff(row, 2 * b)) = pack8(v);
-      *reinterpret_cast<uint4*>(xs + xoff(row, 2 * b + 1)) = pack8(v + 8);
+    for (int i = 0; i < 32; ++i) {
+      const float olo = __shfl_xor_sync(0xFFFFFFFFu, lo2(v[i]), 1);
+      const float ohi = __shfl_xor_sync(0xFFFFFFFFu, hi2(v[i]), 1);
+      v[i] = fma2(sg2, v[i], pk2(olo, ohi));
     }
+  }
+  const float cn = 0.0883883461356163f;        // fp32(1/sqrt(128)) = 0x3DB504F3
+  const uint64_t cn2 = pk2(cn, cn);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = mul2(v[i], cn2);
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    uint64_t blk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) blk[i] = v[8 * b + i];
+    const uint32_t sb = quantize_any(blk, srec, y6, cw[2 * b], cw[2 * b + 1]);
+    sbytes |= sb << (8 * b);
+    write_back_bf16(xs, row, 8 * q + 2 * b, blk);
   }
 }
 
-template <bool ROT, bool TILED, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1)
-    quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,
-                        const __grid_constant__ CUtensorMap tm_pdT, const QParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+// Unrotated path, one thread: the 16-channel block column j = t & 7 of the
+// chunk for rows t/8 + 32 i (i = 0..3), so the block's 8 smooth-factor
+// operand pairs are loaded once for four rows.  NEG selects the negated
+// layout (x / -smooth, written back negated; requires every smooth factor
+// positive) over the sign-fixed one.
+template <bool NEG>
+__device__ __forceinline__ void smooth_cols(uint8_t* xs, const float4* lam4, const float2* srec, float y6, int t,
+                                            uint32_t (&cw)[4][2], uint32_t (&sb)[4]) {
+  const int j = t & 7, r0 = t >> 3;
+  uint64_t nb[8], yb[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 l = lam4[8 * j + i];
+    nb[i] = pk2(l.x, l.y);
+    yb[i] = pk2(l.z, l.w);
+  }
+#pragma unroll
+  for (int rr = 0; rr < 4; ++rr) {
+    const int row = r0 + 32 * rr;
+    const uint4 p0 = *reinterpret_cast<const uint4*>(xs + xoff(row, 2 * j));
+    const uint4 p1 = *reinterpret_cast<const uint4*>(xs + xoff(row, 2 * j + 1));
+    const uint32_t xin[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    uint64_t v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      v[i] = NEG ? div_mk2(bf16x2_to_f2(xin[i]), nb[i], yb[i]) : div_rn2(bf16x2_to_f2(xin[i]), nb[i], yb[i]);
+    const float amax = amax8(v);
+    if (amax < 3.0e38f) {
+      sb[rr] = quant_block<NEG>(v, amax, srec, y6, cw[rr][0], cw[rr][1]);
+    } else {                           // overflow / NaN (rare): redo with the divide unit
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float s0 = NEG ? lo2(nb[i]) : -lo2(nb[i]), s1 = NEG ? hi2(nb[i]) : -hi2(nb[i]);
+        v[i] = pk2(__fdiv_rn(__uint_as_float(xin[i] << 16), s0), __fdiv_rn(__uint_as_float(xin[i] & 0xFFFF0000u), s1));
+      }
+      sb[rr] = quant_block_slow(v, cw[rr][0], cw[rr][1]);
+      if (NEG) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] ^= 0x8000000080000000ull;   // write back -x_hat
+      }
+    }
+    write_back_bf16(xs, row, 2 * j, v);
+  }
+}
+
+template <bool TILED>
+__device__ __forceinline__ void store_cols(const QParams& p, int m0, int t, int kc, const uint32_t (&cw)[4][2],
+                                           const uint32_t (&sb)[4]) {
+  const int j = t & 7, r0 = t >> 3;
+  const int k = kc + 16 * j;
+  if (k >= p.k_limit) return;
+#pragma unroll
+  for (int rr = 0; rr < 4; ++rr) {
+    const int row = r0 + 32 * rr, m = m0 + row;
+    if (m >= p.M) continue;
+    *reinterpret_cast<uint2*>(p.codes + (size_t)m * p.codes_pitch + (k >> 1)) = make_uint2(cw[rr][0], cw[rr][1]);
+    if (TILED) {
+      uint8_t* atom = p.scales + ((size_t)(m >> 7) * p.ka_pad + (k >> 6)) * kSfRepBytes + sf_atom_offset(row, j & 3);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) atom[r * kSfAtomBytes] = (uint8_t)sb[rr];
+    } else
+      p.scales[(size_t)m * p.scales_pitch + (k >> 4)] = (uint8_t)sb[rr];
+  }
+}
+
+template <bool ROT, bool NEG, bool TILED>
+__global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
+    quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_pdT,
+                        const QParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // Round up to 1024 bytes by pointer arithmetic on the __shared__ array, so
+  // every access below stays a shared-memory access (an integer round trip
+  // would turn them into generic ones).
+  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int R = p.R;
   const int pd_stage_bytes = R * kChunk * 2;     // two 64-wide boxes of R rows x 128 B
   uint8_t* X = base;
-  uint8_t* PD = X + STAGES * kXStageBytes;
-  uint8_t* LAM = PD + STAGES * pd_stage_bytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(LAM + STAGES * kLamStageBytes);
+  uint8_t* PD = X + kStages * kXStageBytes;
+  uint8_t* LAM = PD + kStages * pd_stage_bytes;
+  Tables* tabs = reinterpret_cast<Tables*>(LAM + kStages * kLamStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(tabs + 1);
   uint64_t* full = bars;                    // TMA landed
-  uint64_t* xready = bars + STAGES;         // x_hat written back (128 arrivals)
-  uint64_t* empty = bars + 2 * STAGES;      // MMA finished reading the stage
-  uint64_t* done = bars + 3 * STAGES;       // all MMAs of this CTA finished
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 1);
+  uint64_t* xready = bars + kStages;        // x_hat written back (256 arrivals)
+  uint64_t* empty = bars + 2 * kStages;     // MMA finished reading the stage
+  uint64_t* done = bars + 3 * kStages;      // all MMAs of this CTA finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -183,16 +436,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_cols = R <= 32 ? 32u : (R <= 64 ? 64u : 128u);
 
   if (tid == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&xready[s]), kRows);
+      mbar_init(smem_u32(&xready[s]), kComputeThreads);
       mbar_init(smem_u32(&empty[s]), 1);
     }
     mbar_init(smem_u32(done), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (tid < 128) {
+    const float s = e4m3_to_f32((uint32_t)tid);
+    const float r = tid ? __frcp_rn(s) : 0.0f;
+    tabs->srec[tid] = NEG ? make_float2(s, -r) : make_float2(-s, r);   // {-B, RN(1/B)}, B = -+s
+  }
+  if (warp == kProducerWarp) {
     tmem_alloc(smem_u32(tmem_slot), tmem_cols);
     tmem_relinquish();
     if (lane == 0) {
@@ -206,12 +464,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   int issued = 0;   // producer: loads issued
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     if (lane == 0) {
       for (int i = 0; i < nch; ++i) {
-        const int s = i % STAGES;
-        if (i >= STAGES &&
-            !wait_bounded(smem_u32(&empty[s]), ((i / STAGES) - 1) & 1, abort_flag, p.err, kErrQuantTimeout))
+        const int s = i % kStages;
+        if (i >= kStages &&
+            !wait_bounded(smem_u32(&empty[s]), ((i / kStages) - 1) & 1, abort_flag, p.err, kErrQuantTimeout))
           break;
         const int kc = (c_begin + i) * kChunk;
         const uint32_t fb = smem_u32(&full[s]);
@@ -222,17 +480,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(smem_u32(xs + kXBoxBytes), &tm_x, fb, kc + 64, m0);
         tma_load_2d(smem_u32(pds), &tm_pdT, fb, kc, 0);
         tma_load_2d(smem_u32(pds + R * 128), &tm_pdT, fb, kc + 64, 0);
-        bulk_load(smem_u32(LAM + s * kLamStageBytes), p.lam2 + kc, kLamStageBytes, fb);
+        bulk_load(smem_u32(LAM + s * kLamStageBytes), p.lam4 + kc / 2, kLamStageBytes, fb);
         issued = i + 1;
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, (uint32_t)R);
       for (int i = 0; i < nch; ++i) {
-        const int s = i % STAGES;
-        const uint32_t par = (i / STAGES) & 1;
+        const int s = i % kStages;
+        const uint32_t par = (i / kStages) & 1;
         if (!wait_bounded(smem_u32(&full[s]), par, abort_flag, p.err, kErrQuantTimeout)) break;
         if (!wait_bounded(smem_u32(&xready[s]), par, abort_flag, p.err, kErrQuantTimeout)) break;
         tc_fence_after_sync();
@@ -252,31 +510,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // warps 0-3: one thread per token row
-    const int row = tid;
-    const int m = m0 + row;
+    // warps 0-7: the chunk's 128 rows x 128 channels
+    const float y6 = __frcp_rn(6.0f);
+    const int row2 = tid >> 1, q = tid & 1;      // rotated mapping: two threads per row
     for (int i = 0; i < nch; ++i) {
-      const int s = i % STAGES;
-      if (!wait_bounded(smem_u32(&full[s]), (i / STAGES) & 1, abort_flag, p.err, kErrQuantTimeout)) break;
+      const int s = i % kStages;
+      if (!wait_bounded(smem_u32(&full[s]), (i / kStages) & 1, abort_flag, p.err, kErrQuantTimeout)) break;
       const int kc = (c_begin + i) * kChunk;
-      process_chunk<ROT, TILED>(p, X + s * kXStageBytes,
-                                reinterpret_cast<const float2*>(LAM + s * kLamStageBytes), row, m, kc);
-      fence_proxy_async_smem();
-      mbar_arrive(smem_u32(&xready[s]));
+      uint8_t* xs = X + s * kXStageBytes;
+      const float4* lam = reinterpret_cast<const float4*>(LAM + s * kLamStageBytes);
+      if (ROT) {
+        uint32_t cw[8], sbytes;
+        rotate_half(xs, lam, tabs->srec, y6, row2, q, cw, sbytes);
+        fence_proxy_async_smem();
+        mbar_arrive(smem_u32(&xready[s]));
+        const int m = m0 + row2, k0 = kc + 64 * q;
+        if (m < p.M && k0 < p.k_limit) {
+          store_codes<TILED>(p, m, k0, cw);
+          store_scales<TILED>(p, m, row2, k0, sbytes);
+        }
+      } else {
+        uint32_t cw[4][2], sb[4];
+        smooth_cols<NEG>(xs, lam, tabs->srec, y6, tid, cw, sb);
+        fence_proxy_async_smem();
+        mbar_arrive(smem_u32(&xready[s]));
+        store_cols<TILED>(p, m0, tid, kc, cw, sb);
+      }
     }
     // The CTA that owns the last chunk zero-fills the scale atoms beyond Kp
     // (the GEMM's last K tile reads them and they must be finite).
-    if (TILED && m < p.M && c_begin + nch == p.n_chunks) {
-      for (int ka = p.Kp / 64; ka < p.ka_pad; ++ka)
-        *reinterpret_cast<uint32_t*>(p.scales + ((size_t)(m >> 7) * p.ka_pad + ka) * kSfAtomBytes +
-                                     sf_atom_offset(row, 0)) = 0u;
+    if (TILED && tid < kRows && m0 + tid < p.M && c_begin + nch == p.n_chunks) {
+      for (int ka = p.Kp / 64; ka < p.ka_pad; ++ka) {
+        uint8_t* atom = p.scales + ((size_t)((m0 + tid) >> 7) * p.ka_pad + ka) * kSfRepBytes + sf_atom_offset(tid, 0);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) *reinterpret_cast<uint32_t*>(atom + r * kSfAtomBytes) = 0u;
+      }
     }
   }
 
   // ---- rank-R down-projection: TMEM -> L (cluster reduction when K is split)
   const bool want_lr = p.lowrank != nullptr;
-  float* partial = reinterpret_cast<float*>(base);   // reuses the x ring once all MMAs are done
+  const int pstride = R + 4;                          // padded row stride (floats) of the partial tile
+  float* partial = reinterpret_cast<float*>(base);   // reuses the x / proj_down ring once all MMAs are done
   if (want_lr && tid < kRows) {
+    // warps 0-3 read TMEM lane quadrants 0-3: thread tid owns row tid.
     const bool ok = wait_bounded(smem_u32(done), 0, abort_flag, p.err, kErrQuantTimeout);
     tc_fence_after_sync();
     const int row = tid, m = m0 + row;
@@ -285,65 +562,90 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t r[16];
         tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)j, r);
         tmem_ld_wait();
+        if (NEG) {                     // the negated layout accumulated -L
+#pragma unroll
+          for (int t = 0; t < 16; ++t) r[t] ^= 0x80000000u;
+        }
         if (p.ksplit == 1) {
           if (m < p.M) {
             uint4* dst = reinterpret_cast<uint4*>(p.lowrank + (size_t)m * R + j);
-            float f[16];
-#pragma unroll
-            for (int t = 0; t < 16; ++t) f[t] = __uint_as_float(r[t]);
-            dst[0] = pack8(f);
-            dst[1] = pack8(f + 8);
+            dst[0] = make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                                pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                                pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                                pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
+            dst[1] = make_uint4(pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9])),
+                                pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11])),
+                                pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13])),
+                                pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15])));
           }
         } else {
+          float4* dst = reinterpret_cast<float4*>(partial + row * pstride + j);
 #pragma unroll
-          for (int t = 0; t < 16; ++t) partial[row * R + j + t] = __uint_as_float(r[t]);
+          for (int t = 0; t < 4; ++t)
+            dst[t] = make_float4(__uint_as_float(r[4 * t]), __uint_as_float(r[4 * t + 1]),
+                                 __uint_as_float(r[4 * t + 2]), __uint_as_float(r[4 * t + 3]));
         }
       }
     }
   }
   if (want_lr && p.ksplit > 1) {
     cluster_sync();
-    if (tid < kRows && !*abort_flag) {
+    if (tid < kComputeThreads && !*abort_flag) {
+      // Rank r reduces rows [r * 128/ksplit, (r+1) * 128/ksplit) over all
+      // ranks (rank order fixed), four columns per step.
       const uint32_t rank = cluster_ctarank();
       const int rows_per = kRows / p.ksplit;
+      const int r4 = R / 4;
       const uint32_t pbase = smem_u32(partial);
-      for (int idx = tid; idx < rows_per * R; idx += kRows) {
-        const int row = (int)rank * rows_per + idx / R, col = idx % R;
+      for (int idx = tid; idx < rows_per * r4; idx += kComputeThreads) {
+        const int row = (int)rank * rows_per + idx / r4, col = 4 * (idx % r4);
         const int m = m0 + row;
         if (m >= p.M) continue;
-        float acc = 0.0f;
-        for (int q = 0; q < p.ksplit; ++q)
-          acc += ld_shared_cluster_f32(mapa_shared(pbase + (uint32_t)((row * R + col) * 4), (uint32_t)q));
-        p.lowrank[(size_t)m * R + col] = __float2bfloat16_rn(acc);
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        const uint32_t off = (uint32_t)((row * pstride + col) * 4);
+        for (int qr = 0; qr < p.ksplit; ++qr) {
+          const uint32_t ra = mapa_shared(pbase + off, (uint32_t)qr);
+          a0 += ld_shared_cluster_f32(ra);
+          a1 += ld_shared_cluster_f32(ra + 4);
+          a2 += ld_shared_cluster_f32(ra + 8);
+          a3 += ld_shared_cluster_f32(ra + 12);
+        }
+        *reinterpret_cast<uint2*>(p.lowrank + (size_t)m * R + col) =
+            make_uint2(pack_bf16x2(a0, a1), pack_bf16x2(a2, a3));
       }
     }
     cluster_sync();
   }
 
   // ---- cleanup: after an abort, wait (bounded) for the copies this CTA started.
-  if (warp == 4 && lane == 0 && *abort_flag) {
-    for (int s = 0; s < STAGES && s < issued; ++s) {
-      const int last = s + ((issued - 1 - s) / STAGES) * STAGES;
-      wait_for(smem_u32(&full[s]), (last / STAGES) & 1, 100000000ull);
+  if (warp == kProducerWarp && lane == 0 && *abort_flag) {
+    for (int s = 0; s < kStages && s < issued; ++s) {
+      const int last = s + ((issued - 1 - s) / kStages) * kStages;
+      wait_for(smem_u32(&full[s]), (last / kStages) & 1, 100000000ull);
     }
   }
-  if (warp == 5 && lane == 0) wait_for(smem_u32(done), 0, kWaitTimeoutNs);
+  if (warp == kMmaWarp && lane == 0) wait_for(smem_u32(done), 0, kWaitTimeoutNs);
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, tmem_cols);
   }
 }
 
-template <bool ROT, bool TILED, int STAGES>
-cudaError_t launch_impl(const QuantLaunch& L, const QParams& p, int ksplit, cudaStream_t stream) {
-  auto kern = quantize_act_kernel<ROT, TILED, STAGES>;
-  const size_t smem = 1024 + (size_t)STAGES * (kXStageBytes + L.R * kChunk * 2 + kLamStageBytes) + 256;
+size_t smem_bytes(int R) {
+  return 1024 + (size_t)kStages * (kXStageBytes + R * kChunk * 2 + kLamStageBytes) + sizeof(Tables) + 256;
+}
+
+template <bool ROT, bool NEG, bool TILED>
+cudaError_t launch_impl(const CUtensorMap& tm_x, const CUtensorMap& tm_pdT, const QParams& p, int row_tiles,
+                        int ksplit, cudaStream_t stream) {
+  auto kern = quantize_act_kernel<ROT, NEG, TILED>;
+  const size_t smem = smem_bytes(p.R);
   cudaError_t e = ensure_smem_limit(kern, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((L.M + kRows - 1) / kRows), (unsigned)ksplit, 1);
+  cfg.gridDim = dim3((unsigned)row_tiles, (unsigned)ksplit, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -354,7 +656,7 @@ cudaError_t launch_impl(const QuantLaunch& L, const QParams& p, int ksplit, cuda
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, L.tm_x, L.tm_pdT, p);
+  return cudaLaunchKernelEx(&cfg, kern, tm_x, tm_pdT, p);
 }
 
 }  // namespace
@@ -362,21 +664,33 @@ cudaError_t launch_impl(const QuantLaunch& L, const QParams& p, int ksplit, cuda
 cudaError_t launch_quantize_act(const QuantLaunch& L, cudaStream_t stream) {
   if (L.M <= 0) return cudaSuccess;
   const int n_chunks = L.Kp / kChunk;
-  // Split K across a cluster so that small-M batches still spread over many SMs.
   const int row_tiles = (L.M + kRows - 1) / kRows;
+  const bool rot = L.rotate_block == 128;
+  // Split K over a cluster until the grid covers the GPU (148 SMs; two CTAs
+  // per SM without rotation, one with).  Every CTA keeps at least one chunk.
+  const int slots = (rot || L.R > 64) ? 148 : 2 * 148;
+  const int max_split = rot ? 4 : 8;
   int ksplit = 1;
-  for (int cand : {8, 4, 2}) {
+  for (int cand = max_split; cand >= 2; cand >>= 1) {
     const int cpc = (n_chunks + cand - 1) / cand;
-    if (cand <= n_chunks && (cand - 1) * cpc < n_chunks && row_tiles * cand <= 4 * 148) {
+    if (cand <= n_chunks && (cand - 1) * cpc < n_chunks && row_tiles * cand <= 2 * slots) {
       ksplit = cand;
       break;
     }
   }
-  if (L.lowrank == nullptr) ksplit = 1;   // no reduction needed: whole rows per CTA are fine too
+  // Tuning override: SVDQ_QUANT_KSPLIT=1|2|4|8 (applied when it keeps every CTA busy).
+  static const int ks_env = [] {
+    const char* e = getenv("SVDQ_QUANT_KSPLIT");
+    return e ? atoi(e) : 0;
+  }();
+  if (ks_env == 1 || ks_env == 2 || ks_env == 4 || ks_env == 8) {
+    const int cpc_env = (n_chunks + ks_env - 1) / ks_env;
+    if (ks_env <= n_chunks && (ks_env - 1) * cpc_env < n_chunks) ksplit = ks_env;
+  }
   const int cpc = (n_chunks + ksplit - 1) / ksplit;
 
   QParams p;
-  p.lam2 = reinterpret_cast<const float2*>(L.lam2);
+  p.lam4 = reinterpret_cast<const float4*>(L.lam4);
   p.codes = L.codes;
   p.scales = L.scales;
   p.lowrank = reinterpret_cast<__nv_bfloat16*>(L.lowrank);
@@ -390,13 +704,17 @@ cudaError_t launch_quantize_act(const QuantLaunch& L, cudaStream_t stream) {
   p.n_chunks = n_chunks;
   p.ksplit = ksplit;
 
-  const bool rot = L.rotate_block == 128;
   if (rot) {
-    return L.tiled_scales ? launch_impl<true, true, 3>(L, p, ksplit, stream)
-                          : launch_impl<true, false, 3>(L, p, ksplit, stream);
+    return L.tiled_scales ? launch_impl<true, false, true>(L.tm_x, L.tm_pdT, p, row_tiles, ksplit, stream)
+                          : launch_impl<true, false, false>(L.tm_x, L.tm_pdT, p, row_tiles, ksplit, stream);
   }
-  return L.tiled_scales ? launch_impl<false, true, 3>(L, p, ksplit, stream)
-                        : launch_impl<false, false, 3>(L, p, ksplit, stream);
+  if (L.lam_positive) {
+    p.lam4 = reinterpret_cast<const float4*>(L.lam4_neg);
+    return L.tiled_scales ? launch_impl<false, true, true>(L.tm_x, L.tm_pdT, p, row_tiles, ksplit, stream)
+                          : launch_impl<false, true, false>(L.tm_x, L.tm_pdT, p, row_tiles, ksplit, stream);
+  }
+  return L.tiled_scales ? launch_impl<false, false, true>(L.tm_x, L.tm_pdT, p, row_tiles, ksplit, stream)
+                        : launch_impl<false, false, false>(L.tm_x, L.tm_pdT, p, row_tiles, ksplit, stream);
 }
 
 }  // namespace svdq

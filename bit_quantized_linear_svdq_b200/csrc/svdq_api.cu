@@ -9,7 +9,7 @@
 #include <mutex>
 #include <string>
 
-#include "../../include/svdq.h"
+#include "svdq.h"
 #include "kcommon.cuh"
 #include "svdq_kernels.h"
 
@@ -17,10 +17,12 @@ struct svdq_linear {
   int device;
   int K, N, R, Kp, ka_pad, k_tiles, rotate_block;
   uint8_t* qw;            // (N, Kp/2) packed E2M1, rows zero-padded to Kp
-  uint8_t* sfb;           // weight scale tiles: ceil(N/128) x ka_pad atoms of 512 bytes
+  uint8_t* sfb;           // weight scale tiles: ceil(N/128) x ka_pad replicated atoms of 2 KB
   __nv_bfloat16* pdT;     // proj_down^T (R, Kp), zero-padded
   __nv_bfloat16* pu;      // proj_up (N, R)
-  float2* lam2;           // (Kp) {smooth, 1/smooth}, padded with {1, 1}
+  float4* lam4;           // (Kp/2) {-s_k, -s_k+1, 1/s_k, 1/s_k+1} per channel pair, padded with s = 1
+  float4* lam4_neg;       // (Kp/2) the same operands for dividing by -s_k
+  bool lam_positive;      // every smooth factor is positive
   float* alpha;           // (roundup(N, 128)) wcscales * wtscale, zero-padded
   unsigned* err;          // device error word
   CUtensorMap tm_b, tm_pdT, tm_pu;
@@ -91,7 +93,9 @@ __global__ void repack_weight_scales(const uint8_t* __restrict__ wscales, uint8_
     const int kb = (int)(i / N), n = (int)(i % N);
     const uint8_t b = wscales[i];
     if ((b & 0x7F) == 0x7F) atomicOr(bad, 1u);       // e4m3 NaN
-    sfb[((size_t)(n >> 7) * ka_pad + (kb >> 2)) * svdq::kSfAtomBytes + svdq::sf_atom_offset(n & 127, kb & 3)] = b;
+    uint8_t* atom = sfb + ((size_t)(n >> 7) * ka_pad + (kb >> 2)) * svdq::kSfRepBytes + svdq::sf_atom_offset(n & 127, kb & 3);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) atom[r * svdq::kSfAtomBytes] = b;
   }
 }
 
@@ -104,16 +108,23 @@ __global__ void transpose_proj_down(const __nv_bfloat16* __restrict__ pd, __nv_b
   }
 }
 
-__global__ void prepare_smooth(const __nv_bfloat16* __restrict__ sf, float2* __restrict__ lam2, int K, int Kp,
-                               unsigned* bad) {
-  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < Kp; k += gridDim.x * blockDim.x) {
-    if (k < K) {
-      const float l = __bfloat162float(sf[k]);
-      if (!(isfinite(l) && l != 0.0f)) atomicOr(bad, 2u);
-      lam2[k] = make_float2(l, __frcp_rn(l));
-    } else {
-      lam2[k] = make_float2(1.0f, 1.0f);
+// Per channel pair (k, k+1): {-s_k, -s_k+1, RN(1/s_k), RN(1/s_k+1)} and its
+// negation, the operands of the quantizer's two-lane correctly rounded
+// division by s or by -s; padding channels get s = 1.  bad bit 2: a zero or
+// non-finite factor; bit 4: a negative one.
+__global__ void prepare_smooth(const __nv_bfloat16* __restrict__ sf, float4* __restrict__ lam4,
+                               float4* __restrict__ lam4_neg, int K, int Kp, unsigned* bad) {
+  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < Kp / 2; j += gridDim.x * blockDim.x) {
+    float l0 = 1.0f, l1 = 1.0f;
+    if (2 * j < K) {                 // K is even, so channel 2j+1 exists too
+      l0 = __bfloat162float(sf[2 * j]);
+      l1 = __bfloat162float(sf[2 * j + 1]);
+      if (!(isfinite(l0) && l0 != 0.0f && isfinite(l1) && l1 != 0.0f)) atomicOr(bad, 2u);
+      if (l0 < 0.0f || l1 < 0.0f) atomicOr(bad, 4u);
     }
+    const float r0 = __frcp_rn(l0), r1 = __frcp_rn(l1);
+    lam4[j] = make_float4(-l0, -l1, r0, r1);
+    lam4_neg[j] = make_float4(l0, l1, -r0, -r1);
   }
 }
 
@@ -148,7 +159,8 @@ void free_handle(svdq_linear* h) {
   cudaFree(h->sfb);
   cudaFree(h->pdT);
   cudaFree(h->pu);
-  cudaFree(h->lam2);
+  cudaFree(h->lam4);
+  cudaFree(h->lam4_neg);
   cudaFree(h->alpha);
   cudaFree(h->err);
   delete h;
@@ -162,7 +174,7 @@ WsLayout ws_layout(const svdq_linear* h, int M) {
   WsLayout w;
   w.codes = 0;
   w.sfa = align256((size_t)M * (h->Kp / 2));
-  w.lr = align256(w.sfa + (size_t)((M + 127) / 128) * h->ka_pad * svdq::kSfAtomBytes);
+  w.lr = align256(w.sfa + (size_t)((M + 127) / 128) * h->ka_pad * svdq::kSfRepBytes);
   w.total = align256(w.lr + (size_t)M * h->R * 2);
   return w;
 }
@@ -238,10 +250,11 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
   } while (0)
 
   CREATE_CUDA(cudaMalloc(&h->qw, (size_t)d->N * (h->Kp / 2)));
-  CREATE_CUDA(cudaMalloc(&h->sfb, (size_t)n_tiles * h->ka_pad * svdq::kSfAtomBytes));
+  CREATE_CUDA(cudaMalloc(&h->sfb, (size_t)n_tiles * h->ka_pad * svdq::kSfRepBytes));
   CREATE_CUDA(cudaMalloc(&h->pdT, (size_t)d->R * h->Kp * 2));
   CREATE_CUDA(cudaMalloc(&h->pu, (size_t)d->N * d->R * 2));
-  CREATE_CUDA(cudaMalloc(&h->lam2, (size_t)h->Kp * sizeof(float2)));
+  CREATE_CUDA(cudaMalloc(&h->lam4, (size_t)(h->Kp / 2) * sizeof(float4)));
+  CREATE_CUDA(cudaMalloc(&h->lam4_neg, (size_t)(h->Kp / 2) * sizeof(float4)));
   CREATE_CUDA(cudaMalloc(&h->alpha, (size_t)Npad * sizeof(float)));
   CREATE_CUDA(cudaMalloc(&h->err, 2 * sizeof(unsigned)));   // [0] device error word, [1] create-time checks
   CREATE_CUDA(cudaMemsetAsync(h->err, 0, 2 * sizeof(unsigned), stream));
@@ -249,7 +262,7 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
   CREATE_CUDA(cudaMemset2DAsync(h->qw, h->Kp / 2, 0, h->Kp / 2, d->N, stream));
   CREATE_CUDA(cudaMemcpy2DAsync(h->qw, h->Kp / 2, d->qweight, d->K / 2, d->K / 2, d->N, cudaMemcpyDeviceToDevice,
                                 stream));
-  CREATE_CUDA(cudaMemsetAsync(h->sfb, 0, (size_t)n_tiles * h->ka_pad * svdq::kSfAtomBytes, stream));
+  CREATE_CUDA(cudaMemsetAsync(h->sfb, 0, (size_t)n_tiles * h->ka_pad * svdq::kSfRepBytes, stream));
   repack_weight_scales<<<grid_for((long long)(d->K / 16) * d->N), 256, 0, stream>>>(
       static_cast<const uint8_t*>(d->wscales), h->sfb, d->K / 16, d->N, h->ka_pad, h->err + 1);
   CREATE_CUDA(cudaGetLastError());
@@ -257,8 +270,8 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
       static_cast<const __nv_bfloat16*>(d->proj_down), h->pdT, d->K, d->R, h->Kp);
   CREATE_CUDA(cudaGetLastError());
   CREATE_CUDA(cudaMemcpyAsync(h->pu, d->proj_up, (size_t)d->N * d->R * 2, cudaMemcpyDeviceToDevice, stream));
-  prepare_smooth<<<grid_for(h->Kp), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(d->smooth_factor), h->lam2,
-                                                       d->K, h->Kp, h->err + 1);
+  prepare_smooth<<<grid_for(h->Kp / 2), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(d->smooth_factor), h->lam4,
+                                                           h->lam4_neg, d->K, h->Kp, h->err + 1);
   CREATE_CUDA(cudaGetLastError());
   prepare_alpha<<<grid_for(Npad), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(d->wcscales),
                                                      static_cast<const __nv_bfloat16*>(d->wtscale), h->alpha, d->N,
@@ -267,10 +280,11 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
   unsigned bad = 0;
   CREATE_CUDA(cudaMemcpyAsync(&bad, h->err + 1, sizeof(unsigned), cudaMemcpyDeviceToHost, stream));
   CREATE_CUDA(cudaStreamSynchronize(stream));
-  if (bad) {
+  if (bad & 3u) {
     g_last_error = (bad & 1u) ? "wscales holds an e4m3 NaN" : "smooth_factor holds a zero or non-finite value";
     return fail(SVDQ_ERR_INVALID_ARG);
   }
+  h->lam_positive = (bad & 4u) == 0;
 #undef CREATE_CUDA
 
   svdq_status s;
@@ -309,7 +323,9 @@ svdq_status svdq_quantize_act(const svdq_linear* h, const void* x, int M, void* 
   if ((s = make_tmap(&q.tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->K, M, (uint64_t)h->K * 2, 64, 128)) != SVDQ_OK)
     return s;
   q.tm_pdT = h->tm_pdT;
-  q.lam2 = h->lam2;
+  q.lam4 = h->lam4;
+  q.lam4_neg = h->lam4_neg;
+  q.lam_positive = h->lam_positive;
   q.codes = static_cast<uint8_t*>(codes);
   q.scales = static_cast<uint8_t*>(scales);
   q.lowrank = lowrank;
@@ -346,7 +362,9 @@ svdq_status forward_quantize(const svdq_linear* h, const void* x, int M, void* w
   if ((s = make_tmap(&q.tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->K, M, (uint64_t)h->K * 2, 64, 128)) != SVDQ_OK)
     return s;
   q.tm_pdT = h->tm_pdT;
-  q.lam2 = h->lam2;
+  q.lam4 = h->lam4;
+  q.lam4_neg = h->lam4_neg;
+  q.lam_positive = h->lam_positive;
   q.codes = ws + w.codes;
   q.scales = ws + w.sfa;
   q.lowrank = ws + w.lr;

@@ -13,7 +13,9 @@ namespace svdq {
 struct QuantLaunch {
   CUtensorMap tm_x;         // x bf16 (M, K): box {64, 128}, 128B swizzle
   CUtensorMap tm_pdT;       // proj_down^T bf16 (R, Kp): box {64, R}, 128B swizzle
-  const void* lam2;         // float2 (Kp): {smooth, 1/smooth}, padded with {1, 1}
+  const void* lam4;         // float4 (Kp/2): {-s_k, -s_k+1, 1/s_k, 1/s_k+1} per channel pair, padded with s = 1
+  const void* lam4_neg;     // float4 (Kp/2): {s_k, s_k+1, -1/s_k, -1/s_k+1} (dividing by -smooth)
+  bool lam_positive;        // every smooth factor > 0: the negated layout may be used
   uint8_t* codes;           // packed codes, row pitch codes_pitch bytes
   uint8_t* scales;          // row-major (pitch scales_pitch) or tensor-core tiles
   void* lowrank;            // bf16 (M, R) or nullptr

@@ -111,11 +111,32 @@ def test_convert_semantics_ties_signed_zero_saturation():
     rows.append([6.0, -0.1, -0.2, 0.1, 0.24, -0.24, 0.26, -0.26] + [0.0] * 8 + [1e4] + [1.0] * 15 + [0.0] * 32)
     rows.append([0.0] * 16 + [1e-4] * 16 + [-3e-3] + [0.0] * 15 + [448.0 * 6] + [-1.0] * 15)
     rows.append([float(v) for v in np.linspace(-7, 7, K)])
+    rows[3][5] = -0.0            # signed zeros inside blocks with a nonzero scale
+    rows[3][40] = -0.0
+    rows[0][15] = -0.0
     x = np.array(rows, dtype=np.float32)
     bits = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     ck = synthetic.make_checkpoint(4, K, 16, 16, seed=0, n_outliers=0)
     ck.x = bits
     ck.smooth_factor = torch.ones(K).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    layer = make_layer(ck)
+    check_quantizer(layer, ck)
+    check_forward(layer, ck)
+    # Same blocks with some negative smooth factors (the sign-fixed division path).
+    lam = np.ones(K, dtype=np.float32)
+    lam[1::3] = -1.0
+    lam[7] = -0.5
+    ck.smooth_factor = torch.from_numpy(lam).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    layer2 = make_layer(ck)
+    check_quantizer(layer2, ck)
+    check_forward(layer2, ck)
+
+
+def test_negative_smooth_factors_random():
+    ck = synthetic.make_checkpoint(150, 512, 256, 32, seed=12, name="negative_smooth")
+    lam = O.bf16_to_f32(ck.smooth_factor).copy()
+    lam[::5] *= -1.0
+    ck.smooth_factor = torch.from_numpy(lam).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     layer = make_layer(ck)
     check_quantizer(layer, ck)
     check_forward(layer, ck)
