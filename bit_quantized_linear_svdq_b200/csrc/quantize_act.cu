@@ -53,6 +53,11 @@ constexpr int kStages = 2;
 constexpr int kXStageBytes = kRows * kChunk * 2;   // 32 KB: two 64-wide swizzled boxes
 constexpr int kXBoxBytes = kXStageBytes / 2;       // 16 KB
 constexpr int kLamStageBytes = kChunk * 8;         // float4 {-s0,-s1,1/s0,1/s1} per channel pair
+// Forward-layout outputs of one chunk are staged in shared memory and written
+// with one TMA tensor store (codes, 128 rows x 64 bytes) and bulk copies (the
+// chunk's two scale atoms, each to its four replicas).
+constexpr int kCodeStageBytes = kRows * kChunk / 2;   // 8 KB
+constexpr int kSfStageBytes = 2 * kSfAtomBytes;       // 1 KB
 constexpr int kComputeThreads = 256;
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kThreads = 320;
@@ -386,6 +391,27 @@ __device__ __forceinline__ void smooth_cols(uint8_t* xs, const float4* lam4, con
   }
 }
 
+// Stage the chunk's codes and compact scale atoms of the column mapping.
+__device__ __forceinline__ void stage_cols(uint8_t* cst, uint8_t* sst, int t, const uint32_t (&cw)[4][2],
+                                           const uint32_t (&sb)[4]) {
+  const int j = t & 7, r0 = t >> 3;
+#pragma unroll
+  for (int rr = 0; rr < 4; ++rr) {
+    const int row = r0 + 32 * rr;
+    *reinterpret_cast<uint2*>(cst + row * (kChunk / 2) + j * 8) = make_uint2(cw[rr][0], cw[rr][1]);
+    sst[(j >> 2) * kSfAtomBytes + sf_atom_offset(row, j & 3)] = (uint8_t)sb[rr];
+  }
+}
+
+// Stage the chunk's codes and compact scale atoms of the rotated mapping.
+__device__ __forceinline__ void stage_half(uint8_t* cst, uint8_t* sst, int row, int q, const uint32_t (&cw)[8],
+                                           uint32_t sbytes) {
+  uint4* c = reinterpret_cast<uint4*>(cst + row * (kChunk / 2) + q * 32);
+  c[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+  c[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+  *reinterpret_cast<uint32_t*>(sst + q * kSfAtomBytes + sf_atom_offset(row, 0)) = sbytes;
+}
+
 template <bool TILED>
 __device__ __forceinline__ void store_cols(const QParams& p, int m0, int t, int kc, const uint32_t (&cw)[4][2],
                                            const uint32_t (&sb)[4]) {
@@ -409,7 +435,7 @@ __device__ __forceinline__ void store_cols(const QParams& p, int m0, int t, int 
 template <bool ROT, bool NEG, bool TILED>
 __global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
     quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_pdT,
-                        const QParams p) {
+                        const __grid_constant__ CUtensorMap tm_codes, const QParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // Round up to 1024 bytes by pointer arithmetic on the __shared__ array, so
   // every access below stays a shared-memory access (an integer round trip
@@ -420,7 +446,9 @@ __global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
   uint8_t* X = base;
   uint8_t* PD = X + kStages * kXStageBytes;
   uint8_t* LAM = PD + kStages * pd_stage_bytes;
-  Tables* tabs = reinterpret_cast<Tables*>(LAM + kStages * kLamStageBytes);
+  uint8_t* CST = LAM + kStages * kLamStageBytes;       // code staging, one per stage
+  uint8_t* SST = CST + kStages * kCodeStageBytes;      // scale-atom staging, one per stage
+  Tables* tabs = reinterpret_cast<Tables*>(SST + kStages * kSfStageBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(tabs + 1);
   uint64_t* full = bars;                    // TMA landed
   uint64_t* xready = bars + kStages;        // x_hat written back (256 arrivals)
@@ -456,6 +484,7 @@ __global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
     if (lane == 0) {
       prefetch_tmap(&tm_x);
       prefetch_tmap(&tm_pdT);
+      if (TILED) prefetch_tmap(&tm_codes);
     }
   }
   tc_fence_before_sync();
@@ -519,24 +548,50 @@ __global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
       const int kc = (c_begin + i) * kChunk;
       uint8_t* xs = X + s * kXStageBytes;
       const float4* lam = reinterpret_cast<const float4*>(LAM + s * kLamStageBytes);
-      if (ROT) {
-        uint32_t cw[8], sbytes;
-        rotate_half(xs, lam, tabs->srec, y6, row2, q, cw, sbytes);
-        fence_proxy_async_smem();
-        mbar_arrive(smem_u32(&xready[s]));
+      uint32_t cw8[8], sbytes = 0;                 // rotated mapping
+      uint32_t cw[4][2], sb[4];                    // column mapping
+      if (ROT)
+        rotate_half(xs, lam, tabs->srec, y6, row2, q, cw8, sbytes);
+      else
+        smooth_cols<NEG>(xs, lam, tabs->srec, y6, tid, cw, sb);
+      if (TILED) {
+        // The staging buffer of this stage was last read by the stores of
+        // chunk i - 2; tid 0 waits for them, the barrier tells everyone.
+        if (tid == 0) bulk_wait_read<1>();
+        named_bar(1, kComputeThreads);
+        uint8_t* cst = CST + s * kCodeStageBytes;
+        uint8_t* sst = SST + s * kSfStageBytes;
+        if (ROT)
+          stage_half(cst, sst, row2, q, cw8, sbytes);
+        else
+          stage_cols(cst, sst, tid, cw, sb);
+      }
+      fence_proxy_async_smem();                    // x_hat (and staging) -> async proxy
+      mbar_arrive(smem_u32(&xready[s]));
+      if (TILED) {
+        named_bar(1, kComputeThreads);
+        if (tid == 0) {
+          tma_store_2d(&tm_codes, smem_u32(CST + s * kCodeStageBytes), kc / 2, m0);
+          uint8_t* dst = p.scales + ((size_t)blockIdx.x * p.ka_pad + kc / 64) * kSfRepBytes;
+#pragma unroll
+          for (int a = 0; a < 2; ++a)
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+              bulk_store(dst + a * kSfRepBytes + r * kSfAtomBytes, smem_u32(SST + s * kSfStageBytes + a * kSfAtomBytes),
+                         kSfAtomBytes);
+          bulk_commit();
+        }
+      } else if (ROT) {
         const int m = m0 + row2, k0 = kc + 64 * q;
         if (m < p.M && k0 < p.k_limit) {
-          store_codes<TILED>(p, m, k0, cw);
-          store_scales<TILED>(p, m, row2, k0, sbytes);
+          store_codes<false>(p, m, k0, cw8);
+          store_scales<false>(p, m, row2, k0, sbytes);
         }
       } else {
-        uint32_t cw[4][2], sb[4];
-        smooth_cols<NEG>(xs, lam, tabs->srec, y6, tid, cw, sb);
-        fence_proxy_async_smem();
-        mbar_arrive(smem_u32(&xready[s]));
-        store_cols<TILED>(p, m0, tid, kc, cw, sb);
+        store_cols<false>(p, m0, tid, kc, cw, sb);
       }
     }
+    if (TILED && tid == 0) bulk_wait<0>();
     // The CTA that owns the last chunk zero-fills the scale atoms beyond Kp
     // (the GEMM's last K tile reads them and they must be finite).
     if (TILED && tid < kRows && m0 + tid < p.M && c_begin + nch == p.n_chunks) {
@@ -601,14 +656,20 @@ __global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
         const int row = (int)rank * rows_per + idx / r4, col = 4 * (idx % r4);
         const int m = m0 + row;
         if (m >= p.M) continue;
+        const uint32_t off = pbase + (uint32_t)((row * pstride + col) * 4);
+        float4 v[8];
+#pragma unroll
+        for (int qr = 0; qr < 8; ++qr)
+          if (qr < p.ksplit) v[qr] = ld_shared_cluster_v4(mapa_shared(off, (uint32_t)qr));
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-        const uint32_t off = (uint32_t)((row * pstride + col) * 4);
-        for (int qr = 0; qr < p.ksplit; ++qr) {
-          const uint32_t ra = mapa_shared(pbase + off, (uint32_t)qr);
-          a0 += ld_shared_cluster_f32(ra);
-          a1 += ld_shared_cluster_f32(ra + 4);
-          a2 += ld_shared_cluster_f32(ra + 8);
-          a3 += ld_shared_cluster_f32(ra + 12);
+#pragma unroll
+        for (int qr = 0; qr < 8; ++qr) {
+          if (qr < p.ksplit) {
+            a0 += v[qr].x;
+            a1 += v[qr].y;
+            a2 += v[qr].z;
+            a3 += v[qr].w;
+          }
         }
         *reinterpret_cast<uint2*>(p.lowrank + (size_t)m * R + col) =
             make_uint2(pack_bf16x2(a0, a1), pack_bf16x2(a2, a3));
@@ -634,12 +695,13 @@ __global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
 }
 
 size_t smem_bytes(int R) {
-  return 1024 + (size_t)kStages * (kXStageBytes + R * kChunk * 2 + kLamStageBytes) + sizeof(Tables) + 256;
+  return 1024 + (size_t)kStages * (kXStageBytes + R * kChunk * 2 + kLamStageBytes + kCodeStageBytes + kSfStageBytes) +
+         sizeof(Tables) + 256;
 }
 
 template <bool ROT, bool NEG, bool TILED>
-cudaError_t launch_impl(const CUtensorMap& tm_x, const CUtensorMap& tm_pdT, const QParams& p, int row_tiles,
-                        int ksplit, cudaStream_t stream) {
+cudaError_t launch_impl(const CUtensorMap& tm_x, const CUtensorMap& tm_pdT, const CUtensorMap& tm_codes,
+                        const QParams& p, int row_tiles, int ksplit, cudaStream_t stream) {
   auto kern = quantize_act_kernel<ROT, NEG, TILED>;
   const size_t smem = smem_bytes(p.R);
   cudaError_t e = ensure_smem_limit(kern, smem);
@@ -656,7 +718,7 @@ cudaError_t launch_impl(const CUtensorMap& tm_x, const CUtensorMap& tm_pdT, cons
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tm_x, tm_pdT, p);
+  return cudaLaunchKernelEx(&cfg, kern, tm_x, tm_pdT, tm_codes, p);
 }
 
 }  // namespace
@@ -705,16 +767,16 @@ cudaError_t launch_quantize_act(const QuantLaunch& L, cudaStream_t stream) {
   p.ksplit = ksplit;
 
   if (rot) {
-    return L.tiled_scales ? launch_impl<true, false, true>(L.tm_x, L.tm_pdT, p, row_tiles, ksplit, stream)
-                          : launch_impl<true, false, false>(L.tm_x, L.tm_pdT, p, row_tiles, ksplit, stream);
+    return L.tiled_scales ? launch_impl<true, false, true>(L.tm_x, L.tm_pdT, L.tm_codes, p, row_tiles, ksplit, stream)
+                          : launch_impl<true, false, false>(L.tm_x, L.tm_pdT, L.tm_codes, p, row_tiles, ksplit, stream);
   }
   if (L.lam_positive) {
     p.lam4 = reinterpret_cast<const float4*>(L.lam4_neg);
-    return L.tiled_scales ? launch_impl<false, true, true>(L.tm_x, L.tm_pdT, p, row_tiles, ksplit, stream)
-                          : launch_impl<false, true, false>(L.tm_x, L.tm_pdT, p, row_tiles, ksplit, stream);
+    return L.tiled_scales ? launch_impl<false, true, true>(L.tm_x, L.tm_pdT, L.tm_codes, p, row_tiles, ksplit, stream)
+                          : launch_impl<false, true, false>(L.tm_x, L.tm_pdT, L.tm_codes, p, row_tiles, ksplit, stream);
   }
-  return L.tiled_scales ? launch_impl<false, false, true>(L.tm_x, L.tm_pdT, p, row_tiles, ksplit, stream)
-                        : launch_impl<false, false, false>(L.tm_x, L.tm_pdT, p, row_tiles, ksplit, stream);
+  return L.tiled_scales ? launch_impl<false, false, true>(L.tm_x, L.tm_pdT, L.tm_codes, p, row_tiles, ksplit, stream)
+                        : launch_impl<false, false, false>(L.tm_x, L.tm_pdT, L.tm_codes, p, row_tiles, ksplit, stream);
 }
 
 }  // namespace svdq

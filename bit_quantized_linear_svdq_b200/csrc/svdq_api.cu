@@ -60,9 +60,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D row-major tensor map with the 128-byte swizzle; out-of-bounds reads are zero.
+// 2-D row-major tensor map (128-byte swizzle unless stated); out-of-bounds reads are zero,
+// out-of-bounds parts of a stored box are skipped.
 svdq_status make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
-                      uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+                      uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+                      CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) {
     g_last_error = "cuTensorMapEncodeTiled unavailable";
@@ -73,7 +75,7 @@ svdq_status make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, u
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     g_last_error = "cuTensorMapEncodeTiled failed with CUresult " + std::to_string((int)r);
     return SVDQ_ERR_CUDA;
@@ -323,6 +325,7 @@ svdq_status svdq_quantize_act(const svdq_linear* h, const void* x, int M, void* 
   if ((s = make_tmap(&q.tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->K, M, (uint64_t)h->K * 2, 64, 128)) != SVDQ_OK)
     return s;
   q.tm_pdT = h->tm_pdT;
+  q.tm_codes = q.tm_x;   // unused: the public layout is written directly
   q.lam4 = h->lam4;
   q.lam4_neg = h->lam4_neg;
   q.lam_positive = h->lam_positive;
@@ -362,6 +365,9 @@ svdq_status forward_quantize(const svdq_linear* h, const void* x, int M, void* w
   if ((s = make_tmap(&q.tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->K, M, (uint64_t)h->K * 2, 64, 128)) != SVDQ_OK)
     return s;
   q.tm_pdT = h->tm_pdT;
+  if ((s = make_tmap(&q.tm_codes, ws + w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->Kp / 2, M, h->Kp / 2, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_NONE)) != SVDQ_OK)
+    return s;
   q.lam4 = h->lam4;
   q.lam4_neg = h->lam4_neg;
   q.lam_positive = h->lam_positive;

@@ -13,6 +13,7 @@ namespace svdq {
 struct QuantLaunch {
   CUtensorMap tm_x;         // x bf16 (M, K): box {64, 128}, 128B swizzle
   CUtensorMap tm_pdT;       // proj_down^T bf16 (R, Kp): box {64, R}, 128B swizzle
+  CUtensorMap tm_codes;     // tiled_scales only: codes u8 (M, Kp/2): box {64, 128}, no swizzle (TMA store)
   const void* lam4;         // float4 (Kp/2): {-s_k, -s_k+1, 1/s_k, 1/s_k+1} per channel pair, padded with s = 1
   const void* lam4_neg;     // float4 (Kp/2): {s_k, s_k+1, -1/s_k, -1/s_k+1} (dividing by -smooth)
   bool lam_positive;        // every smooth factor > 0: the negated layout may be used

@@ -26,8 +26,8 @@ discrete decision (the 4-bit codes and the e4m3 scales).  Sources:
   worked examples (scale = max|x| / (2^(n-1) - 1) signed, / (2^n - 1)
   unsigned; q = round(x / scale); x_hat = q * scale).
 
-Conventions the pages leave open (each is a reading, listed with reasons in the
-design notes):
+Conventions the pages leave open (each is a reading of them, taken as the
+plainest one the rest of the text supports):
 
 * NVFP4 = E2M1 codes {0, 0.5, 1, 1.5, 2, 3, 4, 6} with a sign bit (bit 3);
   byte j of a row holds element 2j in its low nibble and 2j+1 in its high one.
