@@ -33,6 +33,11 @@ STATUS = {
     0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_SHAPE", 3: "SVDQ_ERR_UNSUPPORTED",
     4: "SVDQ_ERR_CUDA", 5: "SVDQ_ERR_WORKSPACE", 6: "SVDQ_ERR_DEVICE",
 }
+SVDQ_ERR_WORKSPACE = 5
+
+# Size of the fixed per-device scratch array of svdq_linear_forward_noalloc
+# (SVDQ_NOALLOC_SCRATCH_BYTES in the header).
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class SvdqError(RuntimeError):
@@ -80,6 +85,7 @@ def load_library() -> ctypes.CDLL:
         "svdq_linear_forward_host": (ci, [vp, vp, ci, vp, vp, vp, vp, vp]),
         "svdq_linear_forward_quantize": (ci, [vp, vp, ci, vp, vp]),
         "svdq_linear_forward_gemm": (ci, [vp, ci, vp, vp, vp]),
+        "svdq_linear_forward_noalloc": (ci, [vp, vp, ci, vp, vp]),
         "svdq_device_status": (ci, [vp, ctypes.POINTER(ci)]),
         "svdq_status_string": (ctypes.c_char_p, [ci]),
         "svdq_last_error": (ctypes.c_char_p, []),
@@ -167,6 +173,20 @@ def svdq_linear_forward_host(handle, x_host_ptr, M, y_host_ptr, x_dev_ptr, y_dev
     _check(load_library().svdq_linear_forward_host(handle, x_host_ptr, M, y_host_ptr, x_dev_ptr, y_dev_ptr,
                                                    workspace_ptr, _stream(stream)),
            "svdq_linear_forward_host")
+
+
+def svdq_linear_forward_noalloc(handle, x_ptr, M, y_ptr, stream=None) -> None:
+    """The forward pass with its intermediates in the library's fixed per-device
+    scratch array (no workspace argument, nothing allocated): for callers that
+    cannot allocate device memory when they run the layer.  M too large for the
+    array raises SvdqError(SVDQ_ERR_WORKSPACE); calls that can overlap on the
+    GPU share the array and race."""
+    st = load_library().svdq_linear_forward_noalloc(handle, x_ptr, M, y_ptr, _stream(stream))
+    if st == SVDQ_ERR_WORKSPACE:
+        need = svdq_workspace_bytes(handle, M)
+        raise SvdqError(st, f"svdq_linear_forward_noalloc: M={M} needs {need} bytes of scratch, "
+                            f"the fixed array holds {NOALLOC_SCRATCH_BYTES}")
+    _check(st, "svdq_linear_forward_noalloc")
 
 
 def svdq_device_status(handle) -> int:

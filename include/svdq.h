@@ -152,6 +152,34 @@ SVDQ_API svdq_status svdq_linear_forward_host(const svdq_linear* h, const void* 
                                      void* x_dev, void* y_dev, void* workspace, void* stream);
 
 /*
+ * svdq_linear_forward_noalloc -- svdq_linear_forward without a caller
+ * workspace and without allocating anything.  The pages have no counterpart:
+ * this is a library convenience for callers that cannot allocate device memory
+ * when they run the layer -- hosts that pass a kernel its inputs and outputs
+ * but no scratch buffer (plugin interfaces, runtimes that own all device
+ * memory), and latency-bound loops that must not call cudaMalloc, which can
+ * block on and synchronize with work already queued on the device.
+ *   x (M, K) bf16 in, y (M, N) bf16 out: caller-owned device memory, 16-byte
+ *   aligned, exactly as for svdq_linear_forward.
+ * The intermediates go to a library-owned device array of
+ * SVDQ_NOALLOC_SCRATCH_BYTES (32 MiB) per device, held from the first call on
+ * that device until the process exits.  M whose svdq_workspace_bytes(h, M)
+ * exceeds it returns SVDQ_ERR_WORKSPACE before anything is launched (about
+ * 14,000 rows at K = 3072, R = 32); use svdq_linear_forward for larger M.
+ * The first call on each device (made with that device current) looks up the
+ * array's device address and caches it; make that first call before any
+ * stream capture begins.  The call itself allocates and frees nothing.
+ * Every call on a device -- any handle, thread or stream -- shares the one
+ * array, which keeps the previous call's contents: calls whose kernels can
+ * overlap on the GPU race and corrupt each other's results, so order them (one
+ * stream, or events).  Nothing in the array needs to start at zero: every
+ * byte the GEMM reads is written earlier in the same call.
+ */
+#define SVDQ_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+SVDQ_API svdq_status svdq_linear_forward_noalloc(const svdq_linear* h, const void* x, int M, void* y,
+                                                 void* stream);
+
+/*
  * svdq_device_status -- synchronize the handle's device and read + clear its
  * device error word (nonzero when a kernel's bounded wait expired: the kernel
  * then skipped its remaining work, released its tensor memory and returned).

@@ -20,7 +20,8 @@ def test_exports_every_declared_symbol(lib):
     assert set(names) == {
         "svdq_linear_create", "svdq_linear_destroy", "svdq_workspace_bytes", "svdq_quantize_act",
         "svdq_linear_forward", "svdq_linear_forward_host", "svdq_device_status", "svdq_status_string",
-        "svdq_last_error", "svdq_version", "svdq_linear_forward_quantize", "svdq_linear_forward_gemm"}
+        "svdq_last_error", "svdq_version", "svdq_linear_forward_quantize", "svdq_linear_forward_gemm",
+        "svdq_linear_forward_noalloc"}
     for n in names:
         assert hasattr(lib, n), n
 
@@ -63,6 +64,7 @@ def test_null_handle_calls(lib):
     assert lib.svdq_workspace_bytes(None, 16) == 0
     assert lib.svdq_quantize_act(None, 1, 1, 1, 1, None, None) == 1
     assert lib.svdq_linear_forward(None, 1, 1, 1, 1, None) == 1
+    assert lib.svdq_linear_forward_noalloc(None, 1, 1, 1, None) == 1
     assert lib.svdq_linear_create(None, None, None) == 1
     lib.svdq_linear_destroy(None)
 
