@@ -12,18 +12,22 @@
 // output tiles (tile = blockIdx.x + i * gridDim.x, M-tile fastest).
 //   warp 0 lane 0   TMA producer: per K step (256 FP4 elements) the activation
 //                   and weight code tiles (128 rows x 128 swizzled bytes) and
-//                   their scale atoms (bulk copies) into a kStages ring; per
-//                   tile the L and proj_up tiles into a double buffer.
-//   warp 1          owns all 512 TMEM columns; lane 0 copies each stage's
-//                   scale atoms to TMEM (two tcgen05.cp .128x256b per operand;
-//                   a copy costs about the same whatever its size) and issues the
-//                   block-scaled MMAs (M=128, N=128, K=64, UE4M3 per 16) into
-//                   one of two accumulators; after the K loop it issues the
-//                   bf16 MMAs L . proj_up^T (K = R) into the rank-R accumulator.
+//                   their compact scale atoms (bulk copies) into a kStages
+//                   ring; per tile the L and proj_up tiles.
+//   warp 1          owns all 512 TMEM columns; lane 0 issues the block-scaled
+//                   MMAs (M=128, N=128, K=64, UE4M3 per 16) into one of two
+//                   accumulators, then the bf16 MMAs L . proj_up^T (K = R) into
+//                   the rank-R accumulator.
 //   warps 2-5       epilogue of tile i (TMEM -> registers, y = fma(alpha, acc,
 //                   lr) -> bf16 -> global) while the tensor core runs tile i+1.
+//   warps 6-9       scale warps: each writes the stage's scale factors into its
+//                   own 32-lane TMEM sub-partition with tcgen05.st (every
+//                   sub-partition needs all 128 rows' scales).  A register
+//                   store does not occupy the tensor pipe, whereas a
+//                   tcgen05.cp costs that pipe as much as a 128x128x64 MMA.
 // TMEM columns: accumulators [0,128) and [128,256), rank-R accumulator
-// [256,384), scale factors [384,448) (two buffers of A and B, 16 columns each).
+// [256,384), scale factors [384,512) (four buffers of 32 columns: A in
+// +0..15, B in +16..31, 4 columns per K atom).
 // Every wait is bounded; on expiry the CTA records an error, drains what it
 // started, frees TMEM and exits.
 #include <cuda_runtime.h>
@@ -36,18 +40,20 @@ namespace {
 
 constexpr int BM = 128, BN = 128;
 constexpr int kKTileBytes = 128;                 // 256 FP4 elements per row per stage
-constexpr int kStages = 3;
+constexpr int kMaxStages = 5;
 constexpr int kABytes = BM * kKTileBytes;        // 16 KB
 constexpr int kBBytes = BN * kKTileBytes;        // 16 KB
-constexpr int kSfaBytes = 4 * kSfRepBytes;       // 4 replicated K atoms x 128 rows (8 KB)
-constexpr int kSfbBytes = (BN / 128) * 4 * kSfRepBytes;
-constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;   // 48 KB
+constexpr int kSfaBytes = 4 * kSfAtomBytes;      // 4 K atoms x 128 rows (2 KB)
+constexpr int kSfbBytes = 4 * kSfAtomBytes;
+constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;   // 36 KB
 constexpr int kLrAtomBytesA = BM * 128;          // 64 bf16 of R per row
 constexpr int kLrAtomBytesB = BN * 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kEpiWarps = 4;
+constexpr int kSfWarp0 = 6, kSfWarps = 4;
+constexpr int kSfBufs = 4;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColAcc = 0, kColLr = 256, kColSfa = 384, kColSfb = 416;   // SF: 2 buffers x 16
+constexpr uint32_t kColAcc = 0, kColLr = 256, kColSf = 384;
 
 struct GParams {
   const uint8_t* sfa;
@@ -58,6 +64,7 @@ struct GParams {
   int M, N, R, k_tiles, ka_pad;
   int m_tiles, n_tiles;
   int lr_bufs;      // 2 when two L / proj_up tiles fit in shared memory, else 1
+  int stages;       // depth of the K-step ring (4 or 5, as shared memory allows)
 };
 
 __device__ __forceinline__ void tile_coords(const GParams& p, int tile, int& mt, int& nt) {
@@ -77,11 +84,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int RA = (p.R + 63) / 64;              // 64-wide swizzled boxes covering R
   const int lr_buf_bytes = RA * (kLrAtomBytesA + kLrAtomBytesB);
   uint8_t* stages = base;
-  uint8_t* LRB = stages + kStages * kStageBytes;          // lr_bufs x {L tile, proj_up tile}
+  uint8_t* LRB = stages + p.stages * kStageBytes;          // lr_bufs x {L tile, proj_up tile}
   uint64_t* bars = reinterpret_cast<uint64_t*>(LRB + p.lr_bufs * lr_buf_bytes);
-  uint64_t* full = bars;                        // [kStages] TMA landed
-  uint64_t* empty = full + kStages;             // [kStages] MMAs done reading the stage
-  uint64_t* lr_full = empty + kStages;          // [2] L / proj_up tile landed
+  uint64_t* full = bars;                        // [p.stages] TMA landed
+  uint64_t* empty = full + p.stages;             // [p.stages] MMAs done reading the stage
+  uint64_t* sf_full = empty + p.stages;          // [kSfBufs] scale factors of a stage in TMEM
+  uint64_t* lr_full = sf_full + kSfBufs;        // [2] L / proj_up tile landed
   uint64_t* lr_free = lr_full + 2;              // [2] rank-R MMAs done reading the L / proj_up tile
   uint64_t* acc_full = lr_free + 2;             // [2] accumulator (and rank-R accumulator) ready
   uint64_t* acc_free = acc_full + 2;            // [2] epilogue done reading accumulator
@@ -94,10 +102,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_tiles = p.m_tiles * p.n_tiles;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < p.stages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
+    for (int b = 0; b < kSfBufs; ++b) mbar_init(smem_u32(&sf_full[b]), kSfWarps);
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&lr_full[b]), 1);
       mbar_init(smem_u32(&lr_free[b]), 1);
@@ -129,28 +138,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_pu);
       int g = 0;   // k-stage counter across tiles
       int it = 0;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      bool stop = false;
+      for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x, ++it) {
         int mt, nt;
         tile_coords(p, tile, mt, nt);
         const int m0 = mt * BM, n0 = nt * BN;
-        // L / proj_up tile of this output tile.
-        {
-          const int lb = p.lr_bufs == 2 ? (it & 1) : 0;
-          const int use = p.lr_bufs == 2 ? (it >> 1) : it;
-          if (use >= 1 && !wait_bounded(smem_u32(&lr_free[lb]), (use - 1) & 1, abort_flag, p.err, kErrGemmTimeout))
-            break;
-          uint8_t* lt = LRB + lb * lr_buf_bytes;
-          const uint32_t fb = smem_u32(&lr_full[lb]);
-          mbar_arrive_expect_tx(fb, (uint32_t)lr_buf_bytes);
-          for (int a = 0; a < RA; ++a) {
-            tma_load_2d(smem_u32(lt + a * kLrAtomBytesA), &tm_l, fb, 64 * a, m0);
-            tma_load_2d(smem_u32(lt + RA * kLrAtomBytesA + a * kLrAtomBytesB), &tm_pu, fb, 64 * a, n0);
-          }
-          lr_issued = it + 1;
-        }
-        bool stop = false;
         for (int kt = 0; kt < p.k_tiles; ++kt, ++g) {
-          const int s = g % kStages, n = g / kStages;
+          const int s = g % p.stages, n = g / p.stages;
           if (n >= 1 && !wait_bounded(smem_u32(&empty[s]), (n - 1) & 1, abort_flag, p.err, kErrGemmTimeout)) {
             stop = true;
             break;
@@ -161,12 +155,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(smem_u32(st), &tm_a, fb, kt * kKTileBytes, m0);
           tma_load_2d(smem_u32(st + kABytes), &tm_b, fb, kt * kKTileBytes, n0);
           bulk_load(smem_u32(st + kABytes + kBBytes),
-                    p.sfa + ((size_t)mt * p.ka_pad + (size_t)kt * 4) * kSfRepBytes, kSfaBytes, fb);
+                    p.sfa + ((size_t)mt * p.ka_pad + (size_t)kt * 4) * kSfAtomBytes, kSfaBytes, fb);
           bulk_load(smem_u32(st + kABytes + kBBytes + kSfaBytes),
-                    p.sfb + ((size_t)nt * p.ka_pad + (size_t)kt * 4) * kSfRepBytes, kSfbBytes, fb);
+                    p.sfb + ((size_t)nt * p.ka_pad + (size_t)kt * 4) * kSfAtomBytes, kSfbBytes, fb);
           issued = g + 1;
+          if (kt == p.k_tiles - 1) {
+            // L / proj_up tile of this output tile, read after its K loop.  It
+            // is issued behind the tile's last K step so that, with a single
+            // buffer, waiting for the previous tile's rank-R MMAs never holds
+            // back the K-step ring.
+            const int lb = p.lr_bufs == 2 ? (it & 1) : 0;
+            const int use = p.lr_bufs == 2 ? (it >> 1) : it;
+            if (use >= 1 &&
+                !wait_bounded(smem_u32(&lr_free[lb]), (use - 1) & 1, abort_flag, p.err, kErrGemmTimeout)) {
+              stop = true;
+              break;
+            }
+            uint8_t* lt = LRB + lb * lr_buf_bytes;
+            const uint32_t lf = smem_u32(&lr_full[lb]);
+            mbar_arrive_expect_tx(lf, (uint32_t)lr_buf_bytes);
+            for (int a = 0; a < RA; ++a) {
+              tma_load_2d(smem_u32(lt + a * kLrAtomBytesA), &tm_l, lf, 64 * a, m0);
+              tma_load_2d(smem_u32(lt + RA * kLrAtomBytesA + a * kLrAtomBytesB), &tm_pu, lf, 64 * a, n0);
+            }
+            lr_issued = it + 1;
+          }
         }
-        if (stop) break;
       }
     }
     __syncwarp();
@@ -186,27 +200,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after_sync();
         for (int kt = 0; kt < p.k_tiles; ++kt, ++g) {
-          const int s = g % kStages, n = g / kStages;
-          if (!wait_bounded(smem_u32(&full[s]), n & 1, abort_flag, p.err, kErrGemmTimeout)) {
+          const int s = g % p.stages, b = g % kSfBufs;
+          // The scale warps waited for the stage's data before writing its
+          // scale factors, so their arrival also means the stage has landed.
+          if (!wait_bounded(smem_u32(&sf_full[b]), (g / kSfBufs) & 1, abort_flag, p.err, kErrGemmTimeout)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
           const uint32_t st = smem_u32(stages + s * kStageBytes);
-          const uint32_t sfa_col = kColSfa + (uint32_t)(g & 1) * 16u;
-          const uint32_t sfb_col = kColSfb + (uint32_t)(g & 1) * 16u;
-          // Scale factors: one 128 x 256-bit copy per operand and pair of K atoms
-          // (replicated atoms kb and kb+1 are 2 KB apart; columns 4 kb .. 4 kb + 7).
-#pragma unroll
-          for (int kb = 0; kb < 4; kb += 2) {
-            tmem_cp_128x256b(tmem + sfa_col + kb * 4, sdesc_rows32b(st + kABytes + kBBytes + kb * kSfRepBytes, kSfRepBytes));
-            tmem_cp_128x256b(tmem + sfb_col + kb * 4,
-                             sdesc_rows32b(st + kABytes + kBBytes + kSfaBytes + kb * kSfRepBytes, kSfRepBytes));
-          }
+          const uint32_t sf = tmem + kColSf + (uint32_t)b * 32u;
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
             mma_nvfp4(acc, sdesc_kmajor_sw128(st + kb * 32), sdesc_kmajor_sw128(st + kABytes + kb * 32), idesc_main,
-                      tmem + sfa_col + kb * 4, tmem + sfb_col + kb * 4, (kt | kb) != 0);
+                      sf + kb * 4, sf + 16 + kb * 4, (kt | kb) != 0);
           }
           tc_commit(smem_u32(&empty[s]));
         }
@@ -231,6 +238,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
+  } else if (warp >= kSfWarp0) {
+    // Scale warps: stage g's scale atoms -> TMEM buffer g % kSfBufs of this
+    // warp's lane quadrant.  Lane l's 16 bytes of an atom are the four columns
+    // (rows l, l+32, l+64, l+96) of its TMEM lane.
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    int g = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int kt = 0; kt < p.k_tiles; ++kt, ++g) {
+        const int s = g % p.stages, b = g % kSfBufs;
+        // Buffer b was last read by the MMAs of stage g - kSfBufs.  The whole
+        // warp agrees on the outcome before the warp-wide TMEM store.
+        bool w = true;
+        if (g >= kSfBufs)
+          w = wait_bounded(smem_u32(&empty[(g - kSfBufs) % p.stages]), ((g - kSfBufs) / p.stages) & 1, abort_flag,
+                           p.err, kErrGemmTimeout);
+        if (w) w = wait_bounded(smem_u32(&full[s]), (g / p.stages) & 1, abort_flag, p.err, kErrGemmTimeout);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t sfs = smem_u32(stages + s * kStageBytes + kABytes + kBBytes) + lane * 16;
+        uint32_t v[32];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {      // atoms 0..3 of A, then 0..3 of B
+          const uint4 q = ld_shared_v4(sfs + a * kSfAtomBytes);
+          v[4 * a + 0] = q.x;
+          v[4 * a + 1] = q.y;
+          v[4 * a + 2] = q.z;
+          v[4 * a + 3] = q.w;
+        }
+        tmem_st32(lane_base + kColSf + (uint32_t)b * 32u, v);
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sf_full[b]));
+      }
+    }
   } else {
     // Epilogue: warps 2..5 cover TMEM lane quadrants 2, 3, 0, 1.
     const int q = warp & 3;
@@ -242,7 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tile_coords(p, tile, mt, nt);
       const int m = mt * BM + row, n0 = nt * BN;
       const int ab = it & 1;
-      if (!wait_bounded(smem_u32(&acc_full[ab]), (it >> 1) & 1, abort_flag, p.err, kErrGemmTimeout)) break;
+      const bool w = wait_bounded(smem_u32(&acc_full[ab]), (it >> 1) & 1, abort_flag, p.err, kErrGemmTimeout);
+      if (!__all_sync(0xffffffffu, w)) break;
       tc_fence_after_sync();
       const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
@@ -296,9 +343,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- cleanup
   if (warp == 0 && lane == 0 && *abort_flag) {
-    for (int s = 0; s < kStages && s < issued; ++s) {
-      const int last = s + ((issued - 1 - s) / kStages) * kStages;
-      wait_for(smem_u32(&full[s]), (last / kStages) & 1, 100000000ull);
+    for (int s = 0; s < p.stages && s < issued; ++s) {
+      const int last = s + ((issued - 1 - s) / p.stages) * p.stages;
+      wait_for(smem_u32(&full[s]), (last / p.stages) & 1, 100000000ull);
     }
     for (int b = 0; b < p.lr_bufs && b < lr_issued; ++b) {
       const int last_it = b + ((lr_issued - 1 - b) / p.lr_bufs) * p.lr_bufs;
@@ -325,7 +372,12 @@ cudaError_t launch_gemm_nvfp4_lr(const GemmLaunch& L, cudaStream_t stream) {
   if (L.M <= 0) return cudaSuccess;
   const int RA = (L.R + 63) / 64;
   const int lr_buf_bytes = RA * (kLrAtomBytesA + kLrAtomBytesB);
-  const size_t fixed = 1024 + (size_t)kStages * kStageBytes + 256;
+  // Deepest ring that fits beside one L / proj_up buffer; a second buffer
+  // only when the ring keeps its full depth.
+  int stages = kMaxStages;
+  while (stages > 2 && 1024 + (size_t)stages * kStageBytes + 256 + lr_buf_bytes > 227 * 1024) --stages;
+  if (stages < kSfBufs) return cudaErrorInvalidValue;   // the scale warps' buffer reuse needs stages >= kSfBufs
+  const size_t fixed = 1024 + (size_t)stages * kStageBytes + 256;
   const int lr_bufs = (fixed + 2 * (size_t)lr_buf_bytes <= 227 * 1024) ? 2 : 1;
   const size_t smem = fixed + (size_t)lr_bufs * lr_buf_bytes;
   cudaError_t e = ensure_smem_limit(gemm_nvfp4_lr_kernel, smem);
@@ -351,6 +403,7 @@ cudaError_t launch_gemm_nvfp4_lr(const GemmLaunch& L, cudaStream_t stream) {
   p.m_tiles = (L.M + BM - 1) / BM;
   p.n_tiles = (L.N + BN - 1) / BN;
   p.lr_bufs = lr_bufs;
+  p.stages = stages;
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = tiles < num_sms ? tiles : num_sms;
   gemm_nvfp4_lr_kernel<<<grid, kThreads, smem, stream>>>(L.tm_a, L.tm_b, L.tm_l, L.tm_pu, p);

@@ -1,0 +1,421 @@
+// gemm_nvfp4_n256.cu -- block-scaled NVFP4 GEMM with the SVDQuant rank-R
+// correction, 128 x 256 output tiles, for sm_100a tensor cores (tcgen05).
+//
+//   y[m, n] = bf16( alpha'[n] * ( sum_k Q(x_hat)[m, k] Q(W)[n, k] + sum_r L[m, r] proj_up'[n, r] ) )
+//   proj_up'[n, r] = bf16(proj_up[n, r] / alpha[n]),  alpha[n] = wcscales[n] * wtscale
+//
+// ("SVDQuant W4A4", vLLM-Omni svdquant.md: the NVFP4 GEMM followed by the
+// bf16 rank correction of "Runtime support".)  Dividing proj_up by alpha once
+// at create time lets the rank-R product accumulate into the same TMEM
+// accumulator as the main product, which leaves tensor memory for a 256-wide
+// tile: per byte brought into shared memory it does a third more work than a
+// 128 x 128 tile.  Columns whose alpha is zero get alpha' = 1 and all-zero
+// weight scales, so y = L proj_up^T exactly as the layer requires.
+//
+// Persistent kernel, one CTA per SM, static tile schedule (M-tile fastest):
+//   warp 0 lane 0   TMA producer: per K step (256 FP4 elements) the activation
+//                   tile (128 rows) and weight tile (256 rows) of codes and
+//                   their compact scale atoms into a 3-deep ring; per tile the
+//                   L and proj_up' tiles.
+//   warp 1          owns 512 TMEM columns: accumulator [0,256), scale factors
+//                   [256,400) (three buffers of 48 columns: A in +0..15, B in
+//                   +16..47, 8 columns per K atom: rows 0-127 then 128-255).
+//                   Lane 0 issues four MMAs per K step (M=128, N=256, K=64,
+//                   UE4M3 per 16), then the bf16 MMAs L . proj_up'^T (K = R)
+//                   into the same accumulator.
+//   warps 2-5       epilogue: TMEM -> registers, alpha' * acc -> bf16 into a
+//                   128B-swizzled staging tile (conflict-free), TMA stores to y.
+//   warps 6-9       scale warps: tcgen05.st of each stage's scale factors into
+//                   their own 32-lane TMEM sub-partition (off the tensor pipe).
+// Every wait is bounded; on expiry the CTA records an error, drains what it
+// started, frees TMEM and exits.
+#include <cuda_runtime.h>
+
+#include "kcommon.cuh"
+#include "svdq_kernels.h"
+
+namespace svdq {
+namespace {
+
+constexpr int BM = 128, BN = 256;
+constexpr int kKTileBytes = 128;                 // 256 FP4 elements per row per stage
+constexpr int kStages = 3;
+constexpr int kABytes = BM * kKTileBytes;        // 16 KB
+constexpr int kBBytes = BN * kKTileBytes;        // 32 KB
+constexpr int kSfaBytes = 4 * kSfAtomBytes;      // 4 K atoms, 128 rows (2 KB)
+constexpr int kSfbBytes = 2 * 4 * kSfAtomBytes;  // two 128-row halves (4 KB)
+constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;   // 54 KB
+constexpr int kThreads = 320;
+constexpr int kEpiWarps = 4;
+constexpr int kSfWarp0 = 6, kSfWarps = 4;
+constexpr int kSfBufs = kStages;                // the scale warps' buffer reuse needs kStages >= kSfBufs
+constexpr int kSfCols = 48;
+constexpr int kStageOutBytes = 2 * 32 * 128;     // per epilogue warp: 32 rows x 128 columns bf16, two 64-column boxes
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColAcc = 0, kColSf = 256;
+
+struct GParams {
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  const float* alpha;     // alpha' (folded)
+  __nv_bfloat16* y;
+  unsigned* err;
+  int M, N, R, k_tiles, ka_pad;
+  int m_tiles, n_tiles;   // n_tiles of 256 columns
+  int lr_row_bytes;       // bytes per row of the L / proj_up' tiles in shared memory (32 or 64)
+  int y_tma;              // write y through the staging tile and TMA stores
+};
+
+// Shared-memory descriptor for a K-major bf16 tile with 32/64/128-byte rows
+// (the matching swizzle), 8-row groups 8 * row_bytes apart.
+__device__ __forceinline__ uint64_t sdesc_kmajor_rows(uint32_t saddr, int row_bytes) {
+  const uint64_t layout = row_bytes == 128 ? 2ull : (row_bytes == 64 ? 4ull : 6ull);
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(16u >> 4) << 16) |
+         ((uint64_t)((8u * (uint32_t)row_bytes) >> 4) << 32) | (1ull << 46) | (layout << 61);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_nvfp4_n256_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                           const __grid_constant__ CUtensorMap tm_l, const __grid_constant__ CUtensorMap tm_pu,
+                           const __grid_constant__ CUtensorMap tm_y, const GParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int lr_l_bytes = BM * p.lr_row_bytes, lr_buf_bytes = (BM + BN) * p.lr_row_bytes;
+  uint8_t* stages = base;
+  uint8_t* OUT = stages + kStages * kStageBytes;                // kEpiWarps x kStageOutBytes
+  uint8_t* LRB = OUT + kEpiWarps * kStageOutBytes;              // one {L tile, proj_up' tile}
+  uint64_t* bars = reinterpret_cast<uint64_t*>(LRB + lr_buf_bytes);
+  uint64_t* full = bars;                        // [kStages] TMA landed
+  uint64_t* empty = full + kStages;             // [kStages] MMAs done reading the stage
+  uint64_t* sf_full = empty + kStages;          // [kSfBufs] scale factors of a stage in TMEM
+  uint64_t* lr_full = sf_full + kSfBufs;        // [1] L / proj_up' tile landed
+  uint64_t* lr_free = lr_full + 1;              // [1] rank-R MMAs done reading it
+  uint64_t* acc_full = lr_free + 1;             // [1] accumulator ready
+  uint64_t* acc_free = acc_full + 1;            // [1] epilogue done reading the accumulator
+  uint64_t* mma_done = acc_free + 1;            // [1] every MMA of this CTA finished (teardown)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int num_tiles = p.m_tiles * p.n_tiles;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < kSfBufs; ++b) mbar_init(smem_u32(&sf_full[b]), kSfWarps);
+    mbar_init(smem_u32(lr_full), 1);
+    mbar_init(smem_u32(lr_free), 1);
+    mbar_init(smem_u32(acc_full), 1);
+    mbar_init(smem_u32(acc_free), kEpiWarps);
+    mbar_init(smem_u32(mma_done), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  int issued = 0, lr_issued = 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_a);
+      prefetch_tmap(&tm_b);
+      prefetch_tmap(&tm_l);
+      prefetch_tmap(&tm_pu);
+      int g = 0, it = 0;
+      bool stop = false;
+      for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x, ++it) {
+        const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
+        const int m0 = mt * BM, n0 = nt * BN;
+        for (int kt = 0; kt < p.k_tiles; ++kt, ++g) {
+          const int s = g % kStages, n = g / kStages;
+          if (n >= 1 && !wait_bounded(smem_u32(&empty[s]), (n - 1) & 1, abort_flag, p.err, kErrGemmTimeout)) {
+            stop = true;
+            break;
+          }
+          uint8_t* st = stages + s * kStageBytes;
+          const uint32_t fb = smem_u32(&full[s]);
+          mbar_arrive_expect_tx(fb, kStageBytes);
+          tma_load_2d(smem_u32(st), &tm_a, fb, kt * kKTileBytes, m0);
+          tma_load_2d(smem_u32(st + kABytes), &tm_b, fb, kt * kKTileBytes, n0);
+          bulk_load(smem_u32(st + kABytes + kBBytes),
+                    p.sfa + ((size_t)mt * p.ka_pad + (size_t)kt * 4) * kSfAtomBytes, kSfaBytes, fb);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            bulk_load(smem_u32(st + kABytes + kBBytes + kSfaBytes + h * (kSfbBytes / 2)),
+                      p.sfb + ((size_t)(2 * nt + h) * p.ka_pad + (size_t)kt * 4) * kSfAtomBytes, kSfbBytes / 2, fb);
+          issued = g + 1;
+          if (kt == p.k_tiles - 1) {
+            // L / proj_up' tile of this output tile, read after its K loop;
+            // issued behind the last K step so that waiting for the previous
+            // tile's rank-R MMAs never holds back the K-step ring.
+            if (it >= 1 && !wait_bounded(smem_u32(lr_free), (it - 1) & 1, abort_flag, p.err, kErrGemmTimeout)) {
+              stop = true;
+              break;
+            }
+            const uint32_t lf = smem_u32(lr_full);
+            mbar_arrive_expect_tx(lf, (uint32_t)lr_buf_bytes);
+            tma_load_2d(smem_u32(LRB), &tm_l, lf, 0, m0);
+            tma_load_2d(smem_u32(LRB + lr_l_bytes), &tm_pu, lf, 0, n0);
+            lr_issued = it + 1;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc_main = idesc_nvfp4(BM, BN);
+      const uint32_t idesc_lr = idesc_bf16_f32(BM, BN);
+      int g = 0, it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+        if (it >= 1 && !wait_bounded(smem_u32(acc_free), (it - 1) & 1, abort_flag, p.err, kErrGemmTimeout)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        for (int kt = 0; kt < p.k_tiles; ++kt, ++g) {
+          const int s = g % kStages, b = g % kSfBufs;
+          // The scale warps waited for the stage's data before writing its
+          // scale factors, so their arrival also means the stage has landed.
+          if (!wait_bounded(smem_u32(&sf_full[b]), (g / kSfBufs) & 1, abort_flag, p.err, kErrGemmTimeout)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t st = smem_u32(stages + s * kStageBytes);
+          const uint32_t sf = tmem + kColSf + (uint32_t)b * kSfCols;
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb)
+            mma_nvfp4(tmem + kColAcc, sdesc_kmajor_sw128(st + kb * 32), sdesc_kmajor_sw128(st + kABytes + kb * 32),
+                      idesc_main, sf + 4 * kb, sf + 16 + 8 * kb, (kt | kb) != 0);
+          tc_commit(smem_u32(&empty[s]));
+        }
+        if (!ok) break;
+        if (!wait_bounded(smem_u32(lr_full), it & 1, abort_flag, p.err, kErrGemmTimeout)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t la = smem_u32(LRB), pa = la + lr_l_bytes;
+        for (int kk = 0; kk < p.R / 16; ++kk) {
+          // K = 16 bf16 = 32 bytes per MMA inside the (swizzled) row.
+          mma_bf16(tmem + kColAcc, sdesc_kmajor_rows(la + kk * 32, p.lr_row_bytes),
+                   sdesc_kmajor_rows(pa + kk * 32, p.lr_row_bytes), idesc_lr, 1u);
+        }
+        tc_commit(smem_u32(lr_free));
+        tc_commit(smem_u32(acc_full));
+      }
+    }
+    __syncwarp();
+  } else if (warp >= kSfWarp0) {
+    // Scale warps: stage g's scale atoms -> TMEM buffer g % kSfBufs of this
+    // warp's lane quadrant.  Lane l's 16 bytes of an atom are the four columns
+    // (rows l, l+32, l+64, l+96) of its TMEM lane.
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    int g = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int kt = 0; kt < p.k_tiles; ++kt, ++g) {
+        const int s = g % kStages, b = g % kSfBufs;
+        // Buffer b was last read by the MMAs of stage g - kSfBufs.  The whole
+        // warp agrees on the outcome before the warp-wide TMEM stores.
+        bool w = true;
+        if (g >= kSfBufs)
+          w = wait_bounded(smem_u32(&empty[(g - kSfBufs) % kStages]), ((g - kSfBufs) / kStages) & 1, abort_flag,
+                           p.err, kErrGemmTimeout);
+        if (w) w = wait_bounded(smem_u32(&full[s]), (g / kStages) & 1, abort_flag, p.err, kErrGemmTimeout);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t sfs = smem_u32(stages + s * kStageBytes + kABytes + kBBytes) + lane * 16;
+        uint32_t va[32], vb[16];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {      // A atoms -> columns 4a .. 4a+3
+          const uint4 q = ld_shared_v4(sfs + a * kSfAtomBytes);
+          va[4 * a + 0] = q.x;
+          va[4 * a + 1] = q.y;
+          va[4 * a + 2] = q.z;
+          va[4 * a + 3] = q.w;
+        }
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {   // B atom kb: rows 0-127 -> 16+8kb+0..3, rows 128-255 -> +4..7
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint4 q = ld_shared_v4(sfs + kSfaBytes + h * (kSfbBytes / 2) + kb * kSfAtomBytes);
+            const int c = 16 + 8 * kb + 4 * h;   // column in the buffer (a compile-time constant)
+            if (c < 32) {
+              va[c] = q.x;
+              va[c + 1] = q.y;
+              va[c + 2] = q.z;
+              va[c + 3] = q.w;
+            } else {
+              vb[c - 32] = q.x;
+              vb[c - 31] = q.y;
+              vb[c - 30] = q.z;
+              vb[c - 29] = q.w;
+            }
+          }
+        }
+        const uint32_t col = lane_base + kColSf + (uint32_t)b * kSfCols;
+        tmem_st32(col, va);
+        tmem_st16(col + 32, vb);
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sf_full[b]));
+      }
+    }
+  } else {
+    // Epilogue: warps 2..5 cover TMEM lane quadrants 2, 3, 0, 1 (rows 32q..32q+31).
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    uint8_t* out = OUT + (warp - 2) * kStageOutBytes;
+    const uint32_t out_s = smem_u32(out);
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + kColAcc;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
+      const int m0 = mt * BM, n0 = nt * BN, m = m0 + row;
+      const bool w = wait_bounded(smem_u32(acc_full), it & 1, abort_flag, p.err, kErrGemmTimeout);
+      if (!__all_sync(0xffffffffu, w)) break;
+      tc_fence_after_sync();
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        if (p.y_tma) {
+          // The staging tile was last read by the previous half's TMA stores.
+          if (lane == 0) bulk_wait_read<0>();
+          __syncwarp();
+        }
+#pragma unroll 1
+        for (int j = 0; j < 4; ++j) {
+          const int nl = 128 * h + 32 * j;            // first column of this chunk in the tile
+          uint32_t acc[32];
+          tmem_ld32(lane_base + nl, acc);
+          tmem_ld_wait();
+          if (h == 1 && j == 3) {
+            // The whole accumulator has been read: the next tile may start.
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(acc_free));
+          }
+          const float4* al = reinterpret_cast<const float4*>(p.alpha + n0 + nl);
+          uint32_t o[16];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const float4 a4 = __ldg(al + c);
+            o[2 * c] = pack_bf16x2(a4.x * __uint_as_float(acc[4 * c + 0]), a4.y * __uint_as_float(acc[4 * c + 1]));
+            o[2 * c + 1] = pack_bf16x2(a4.z * __uint_as_float(acc[4 * c + 2]), a4.w * __uint_as_float(acc[4 * c + 3]));
+          }
+          if (p.y_tma) {
+            // 128B-swizzled box (64 columns x 32 rows): 16-byte chunk c of row r
+            // at r * 128 + ((c ^ (r & 7)) * 16); this chunk is columns 32 (j & 1) ..
+            const uint32_t box = out_s + (uint32_t)(j >> 1) * 4096u + (uint32_t)lane * 128u;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint32_t chunk = (uint32_t)((j & 1) * 4 + c) ^ (uint32_t)(lane & 7);
+              st_shared_v4(box + chunk * 16u, make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]));
+            }
+          } else if (m < p.M) {
+            __nv_bfloat16* dst = p.y + (size_t)m * p.N + n0 + nl;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              if (n0 + nl + c < p.N) {
+                const uint32_t pr = o[c >> 1];
+                dst[c] = __ushort_as_bfloat16((unsigned short)((c & 1) ? (pr >> 16) : (pr & 0xFFFFu)));
+              }
+            }
+          }
+        }
+        if (p.y_tma) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && m0 + 32 * q < p.M) {
+#pragma unroll
+            for (int bx = 0; bx < 2; ++bx) {
+              const int nc = n0 + 128 * h + 64 * bx;
+              if (nc < p.N) tma_store_2d(&tm_y, out_s + (uint32_t)bx * 4096u, nc, m0 + 32 * q);
+            }
+            bulk_commit();
+          }
+        }
+      }
+    }
+    if (p.y_tma && lane == 0) bulk_wait<0>();
+    __syncwarp();
+  }
+
+  // ---- cleanup
+  if (warp == 0 && lane == 0 && *abort_flag) {
+    for (int s = 0; s < kStages && s < issued; ++s) {
+      const int last = s + ((issued - 1 - s) / kStages) * kStages;
+      wait_for(smem_u32(&full[s]), (last / kStages) & 1, 100000000ull);
+    }
+    if (lr_issued > 0) wait_for(smem_u32(lr_full), (lr_issued - 1) & 1, 100000000ull);
+  }
+  if (warp == 1 && lane == 0) {
+    // No MMA may still be running when the tensor memory is released.
+    tc_commit(smem_u32(mma_done));
+    wait_for(smem_u32(mma_done), 0, kWaitTimeoutNs);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+int gemm_n256_lr_row_bytes(int R) { return R <= 16 ? 32 : 64; }
+
+cudaError_t launch_gemm_nvfp4_n256(const GemmLaunch& L, cudaStream_t stream) {
+  if (L.M <= 0) return cudaSuccess;
+  if (L.R > 32) return cudaErrorInvalidValue;
+  const int row_bytes = gemm_n256_lr_row_bytes(L.R);
+  const size_t smem = 1024 + (size_t)kStages * kStageBytes + (size_t)kEpiWarps * kStageOutBytes +
+                      (size_t)(BM + BN) * row_bytes + 256;
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  cudaError_t e = ensure_smem_limit(gemm_nvfp4_n256_kernel, smem);
+  if (e != cudaSuccess) return e;
+  static int num_sms = 0;
+  if (num_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (num_sms <= 0) num_sms = 148;
+  }
+  GParams p;
+  p.sfa = L.sfa;
+  p.sfb = L.sfb;
+  p.alpha = L.alpha;
+  p.y = reinterpret_cast<__nv_bfloat16*>(L.y);
+  p.err = L.err;
+  p.M = L.M;
+  p.N = L.N;
+  p.R = L.R;
+  p.k_tiles = L.k_tiles;
+  p.ka_pad = L.ka_pad;
+  p.m_tiles = (L.M + BM - 1) / BM;
+  p.n_tiles = (L.N + BN - 1) / BN;
+  p.lr_row_bytes = row_bytes;
+  p.y_tma = L.y_tma ? 1 : 0;
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  gemm_nvfp4_n256_kernel<<<grid, kThreads, smem, stream>>>(L.tm_a, L.tm_b, L.tm_l, L.tm_pu, L.tm_y, p);
+  return cudaGetLastError();
+}
+
+}  // namespace svdq

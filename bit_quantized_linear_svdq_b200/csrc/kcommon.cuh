@@ -25,13 +25,11 @@ constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 // Scale-factor tiles consumed by the block-scaled MMA: for every 128 rows and
 // every 64 K elements (4 scale bytes per row), one 512-byte atom in which the
 // scale of (row r, 16-element block j) sits at byte (r % 32) * 16 + (r / 32) * 4 + j.
-// The MMA reads this atom from every 32-lane TMEM sub-partition, so it is
-// stored four times in a row (a 2 KB "replicated atom": 128 rows x 16 bytes,
-// rows 32q..32q+31 identical), and one tcgen05.cp .128x256b moves two of
-// them (two K atoms) at once.  Replicated atoms are stored K-fastest:
-// (row tile t, K atom a) at (t * ka_pad + a) * 2048.
+// Lane l of a warp thus reads its 16 bytes with one vector load and holds
+// exactly the four TMEM columns (rows l, l+32, l+64, l+96) the MMA expects in
+// TMEM lane l of every 32-lane sub-partition.  Atoms are stored K-fastest:
+// (row tile t, K atom a) at (t * ka_pad + a) * 512.
 constexpr int kSfAtomBytes = 512;
-constexpr int kSfRepBytes = 4 * kSfAtomBytes;
 __host__ __device__ __forceinline__ int sf_atom_offset(int r_in_tile, int j) {
   return (r_in_tile & 31) * 16 + (r_in_tile >> 5) * 4 + j;
 }

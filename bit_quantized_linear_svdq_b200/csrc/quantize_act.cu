@@ -244,9 +244,8 @@ template <bool TILED>
 __device__ __forceinline__ void store_scales(const QParams& p, int m, int row, int k, uint32_t sbytes) {
   // four scale bytes (16-element blocks k/16 .. k/16+3), byte j for block j
   if (TILED) {
-    uint8_t* atom = p.scales + ((size_t)(m >> 7) * p.ka_pad + (k >> 6)) * kSfRepBytes + sf_atom_offset(row, 0);
-#pragma unroll
-    for (int r = 0; r < 4; ++r) *reinterpret_cast<uint32_t*>(atom + r * kSfAtomBytes) = sbytes;
+    uint8_t* atom = p.scales + ((size_t)(m >> 7) * p.ka_pad + (k >> 6)) * kSfAtomBytes + sf_atom_offset(row, 0);
+    *reinterpret_cast<uint32_t*>(atom) = sbytes;
   } else {
     uint8_t* dst = p.scales + (size_t)m * p.scales_pitch + (k >> 4);
     if (k + 64 <= p.k_limit && ((reinterpret_cast<uintptr_t>(dst) & 3u) == 0)) {
@@ -424,9 +423,7 @@ __device__ __forceinline__ void store_cols(const QParams& p, int m0, int t, int 
     if (m >= p.M) continue;
     *reinterpret_cast<uint2*>(p.codes + (size_t)m * p.codes_pitch + (k >> 1)) = make_uint2(cw[rr][0], cw[rr][1]);
     if (TILED) {
-      uint8_t* atom = p.scales + ((size_t)(m >> 7) * p.ka_pad + (k >> 6)) * kSfRepBytes + sf_atom_offset(row, j & 3);
-#pragma unroll
-      for (int r = 0; r < 4; ++r) atom[r * kSfAtomBytes] = (uint8_t)sb[rr];
+      p.scales[((size_t)(m >> 7) * p.ka_pad + (k >> 6)) * kSfAtomBytes + sf_atom_offset(row, j & 3)] = (uint8_t)sb[rr];
     } else
       p.scales[(size_t)m * p.scales_pitch + (k >> 4)] = (uint8_t)sb[rr];
   }
@@ -572,13 +569,9 @@ __global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
         named_bar(1, kComputeThreads);
         if (tid == 0) {
           tma_store_2d(&tm_codes, smem_u32(CST + s * kCodeStageBytes), kc / 2, m0);
-          uint8_t* dst = p.scales + ((size_t)blockIdx.x * p.ka_pad + kc / 64) * kSfRepBytes;
-#pragma unroll
-          for (int a = 0; a < 2; ++a)
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-              bulk_store(dst + a * kSfRepBytes + r * kSfAtomBytes, smem_u32(SST + s * kSfStageBytes + a * kSfAtomBytes),
-                         kSfAtomBytes);
+          // the chunk's two scale atoms are adjacent in the tiled layout
+          bulk_store(p.scales + ((size_t)blockIdx.x * p.ka_pad + kc / 64) * kSfAtomBytes,
+                     smem_u32(SST + s * kSfStageBytes), kSfStageBytes);
           bulk_commit();
         }
       } else if (ROT) {
@@ -596,9 +589,8 @@ __global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
     // (the GEMM's last K tile reads them and they must be finite).
     if (TILED && tid < kRows && m0 + tid < p.M && c_begin + nch == p.n_chunks) {
       for (int ka = p.Kp / 64; ka < p.ka_pad; ++ka) {
-        uint8_t* atom = p.scales + ((size_t)((m0 + tid) >> 7) * p.ka_pad + ka) * kSfRepBytes + sf_atom_offset(tid, 0);
-#pragma unroll
-        for (int r = 0; r < 4; ++r) *reinterpret_cast<uint32_t*>(atom + r * kSfAtomBytes) = 0u;
+        uint8_t* atom = p.scales + ((size_t)((m0 + tid) >> 7) * p.ka_pad + ka) * kSfAtomBytes + sf_atom_offset(tid, 0);
+        *reinterpret_cast<uint32_t*>(atom) = 0u;
       }
     }
   }

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -24,8 +25,13 @@ struct svdq_linear {
   float4* lam4_neg;       // (Kp/2) the same operands for dividing by -s_k
   bool lam_positive;      // every smooth factor is positive
   float* alpha;           // (roundup(N, 128)) wcscales * wtscale, zero-padded
+  __nv_bfloat16* pu_fold; // proj_up' = bf16(proj_up / alpha) (N, R); proj_up where alpha = 0
+  float* alpha_fold;      // (roundup(N, 256)) alpha, or 1 where alpha = 0
+  bool n256;              // GEMM on 128 x 256 tiles with alpha folded into proj_up
+  int lr_row_bytes;       // 128 x 256 GEMM: bytes per row of its L / proj_up' tiles
   unsigned* err;          // device error word
   CUtensorMap tm_b, tm_pdT, tm_pu;
+  CUtensorMap tm_b256, tm_pu_fold;
 };
 
 namespace {
@@ -83,21 +89,28 @@ svdq_status make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, u
   return SVDQ_OK;
 }
 
+CUtensorMapSwizzle lr_swizzle(int row_bytes) {
+  return row_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                         : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ---------------------------------------------------------------- create-time repack kernels
 
-__global__ void repack_weight_scales(const uint8_t* __restrict__ wscales, uint8_t* __restrict__ sfb, int K16, int N,
-                                     int ka_pad, unsigned* bad) {
+// Weight scales into replicated tensor-core atoms.  Columns whose alpha is 0
+// get zero scales: their main product is multiplied by 0 anyway, and a zero
+// there lets the 128 x 256 GEMM give them alpha' = 1 with y = L proj_up^T.
+__global__ void repack_weight_scales(const uint8_t* __restrict__ wscales, const float* __restrict__ alpha,
+                                     uint8_t* __restrict__ sfb, int K16, int N, int ka_pad, unsigned* bad) {
   const long long total = (long long)K16 * N;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
     const int kb = (int)(i / N), n = (int)(i % N);
-    const uint8_t b = wscales[i];
-    if ((b & 0x7F) == 0x7F) atomicOr(bad, 1u);       // e4m3 NaN
-    uint8_t* atom = sfb + ((size_t)(n >> 7) * ka_pad + (kb >> 2)) * svdq::kSfRepBytes + svdq::sf_atom_offset(n & 127, kb & 3);
-#pragma unroll
-    for (int r = 0; r < 4; ++r) atom[r * svdq::kSfAtomBytes] = b;
+    const uint8_t w = wscales[i];
+    if ((w & 0x7F) == 0x7F) atomicOr(bad, 1u);       // e4m3 NaN
+    const uint8_t b = alpha[n] == 0.0f ? 0 : w;
+    sfb[((size_t)(n >> 7) * ka_pad + (kb >> 2)) * svdq::kSfAtomBytes + svdq::sf_atom_offset(n & 127, kb & 3)] = b;
   }
 }
 
@@ -139,6 +152,39 @@ __global__ void prepare_alpha(const __nv_bfloat16* __restrict__ wc, const __nv_b
   }
 }
 
+// alpha' and proj_up' = bf16(proj_up / alpha) for the 128 x 256 GEMM, which
+// computes y = alpha' (acc + L proj_up'^T).  bad bit 8: a column that cannot be
+// folded without leaving the range where the quotient keeps bf16 precision
+// (|alpha| outside [2^-24, 2^24], non-finite values, or a quotient that
+// overflows or falls below the normal range); the layer then uses the
+// 128 x 128 GEMM, which applies alpha in its epilogue.
+__global__ void fold_alpha(const __nv_bfloat16* __restrict__ pu, const float* __restrict__ alpha,
+                           __nv_bfloat16* __restrict__ pu_fold, float* __restrict__ alpha_fold, int N, int R,
+                           int Npad256, unsigned* bad) {
+  const long long total = (long long)Npad256 * R;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
+    const int n = (int)(i / R);
+    const float a = n < N ? alpha[n] : 0.0f;
+    if (i % R == 0) alpha_fold[n] = a == 0.0f ? 1.0f : a;
+    if (n >= N) continue;
+    if (a == 0.0f) {
+      pu_fold[i] = pu[i];
+      continue;
+    }
+    const float fa = fabsf(a);
+    if (!(fa >= 0x1p-24f && fa <= 0x1p24f)) {         // also catches NaN
+      atomicOr(bad, 8u);
+      pu_fold[i] = pu[i];
+      continue;
+    }
+    const float v = __bfloat162float(pu[i]);
+    const __nv_bfloat16 q = __float2bfloat16_rn(__fdiv_rn(v, a));
+    const float qf = __bfloat162float(q);
+    if (!isfinite(qf) || (v != 0.0f && fabsf(qf) < 0x1p-126f)) atomicOr(bad, 8u);
+    pu_fold[i] = q;
+  }
+}
+
 int grid_for(long long n) {
   long long g = (n + 255) / 256;
   return (int)(g < 1 ? 1 : (g > 4096 ? 4096 : g));
@@ -164,6 +210,8 @@ void free_handle(svdq_linear* h) {
   cudaFree(h->lam4);
   cudaFree(h->lam4_neg);
   cudaFree(h->alpha);
+  cudaFree(h->pu_fold);
+  cudaFree(h->alpha_fold);
   cudaFree(h->err);
   delete h;
 }
@@ -176,7 +224,7 @@ WsLayout ws_layout(const svdq_linear* h, int M) {
   WsLayout w;
   w.codes = 0;
   w.sfa = align256((size_t)M * (h->Kp / 2));
-  w.lr = align256(w.sfa + (size_t)((M + 127) / 128) * h->ka_pad * svdq::kSfRepBytes);
+  w.lr = align256(w.sfa + (size_t)((M + 127) / 128) * h->ka_pad * svdq::kSfAtomBytes);
   w.total = align256(w.lr + (size_t)M * h->R * 2);
   return w;
 }
@@ -236,6 +284,8 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
   h->ka_pad = 4 * h->k_tiles;
   const int n_tiles = (d->N + 127) / 128;
   const int Npad = n_tiles * 128;
+  const int n_tiles_even = (n_tiles + 1) & ~1;   // the 128 x 256 GEMM reads scale tiles in pairs
+  const int Npad256 = n_tiles_even * 128;
 
   auto fail = [&](svdq_status s) {
     free_handle(h);
@@ -252,21 +302,27 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
   } while (0)
 
   CREATE_CUDA(cudaMalloc(&h->qw, (size_t)d->N * (h->Kp / 2)));
-  CREATE_CUDA(cudaMalloc(&h->sfb, (size_t)n_tiles * h->ka_pad * svdq::kSfRepBytes));
+  CREATE_CUDA(cudaMalloc(&h->sfb, (size_t)n_tiles_even * h->ka_pad * svdq::kSfAtomBytes));
   CREATE_CUDA(cudaMalloc(&h->pdT, (size_t)d->R * h->Kp * 2));
   CREATE_CUDA(cudaMalloc(&h->pu, (size_t)d->N * d->R * 2));
   CREATE_CUDA(cudaMalloc(&h->lam4, (size_t)(h->Kp / 2) * sizeof(float4)));
   CREATE_CUDA(cudaMalloc(&h->lam4_neg, (size_t)(h->Kp / 2) * sizeof(float4)));
   CREATE_CUDA(cudaMalloc(&h->alpha, (size_t)Npad * sizeof(float)));
+  CREATE_CUDA(cudaMalloc(&h->pu_fold, (size_t)d->N * d->R * 2));
+  CREATE_CUDA(cudaMalloc(&h->alpha_fold, (size_t)Npad256 * sizeof(float)));
   CREATE_CUDA(cudaMalloc(&h->err, 2 * sizeof(unsigned)));   // [0] device error word, [1] create-time checks
   CREATE_CUDA(cudaMemsetAsync(h->err, 0, 2 * sizeof(unsigned), stream));
 
   CREATE_CUDA(cudaMemset2DAsync(h->qw, h->Kp / 2, 0, h->Kp / 2, d->N, stream));
   CREATE_CUDA(cudaMemcpy2DAsync(h->qw, h->Kp / 2, d->qweight, d->K / 2, d->K / 2, d->N, cudaMemcpyDeviceToDevice,
                                 stream));
-  CREATE_CUDA(cudaMemsetAsync(h->sfb, 0, (size_t)n_tiles * h->ka_pad * svdq::kSfRepBytes, stream));
+  CREATE_CUDA(cudaMemsetAsync(h->sfb, 0, (size_t)n_tiles_even * h->ka_pad * svdq::kSfAtomBytes, stream));
+  prepare_alpha<<<grid_for(Npad), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(d->wcscales),
+                                                     static_cast<const __nv_bfloat16*>(d->wtscale), h->alpha, d->N,
+                                                     Npad);
+  CREATE_CUDA(cudaGetLastError());
   repack_weight_scales<<<grid_for((long long)(d->K / 16) * d->N), 256, 0, stream>>>(
-      static_cast<const uint8_t*>(d->wscales), h->sfb, d->K / 16, d->N, h->ka_pad, h->err + 1);
+      static_cast<const uint8_t*>(d->wscales), h->alpha, h->sfb, d->K / 16, d->N, h->ka_pad, h->err + 1);
   CREATE_CUDA(cudaGetLastError());
   transpose_proj_down<<<grid_for((long long)d->R * h->Kp), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(d->proj_down), h->pdT, d->K, d->R, h->Kp);
@@ -275,9 +331,8 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
   prepare_smooth<<<grid_for(h->Kp / 2), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(d->smooth_factor), h->lam4,
                                                            h->lam4_neg, d->K, h->Kp, h->err + 1);
   CREATE_CUDA(cudaGetLastError());
-  prepare_alpha<<<grid_for(Npad), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(d->wcscales),
-                                                     static_cast<const __nv_bfloat16*>(d->wtscale), h->alpha, d->N,
-                                                     Npad);
+  fold_alpha<<<grid_for((long long)Npad256 * d->R), 256, 0, stream>>>(h->pu, h->alpha, h->pu_fold, h->alpha_fold,
+                                                                      d->N, d->R, Npad256, h->err + 1);
   CREATE_CUDA(cudaGetLastError());
   unsigned bad = 0;
   CREATE_CUDA(cudaMemcpyAsync(&bad, h->err + 1, sizeof(unsigned), cudaMemcpyDeviceToHost, stream));
@@ -287,6 +342,14 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
     return fail(SVDQ_ERR_INVALID_ARG);
   }
   h->lam_positive = (bad & 4u) == 0;
+  {
+    // 128 x 256 tiles unless alpha cannot be folded, R > 32, or the
+    // environment asks for the 128 x 128 GEMM (SVDQ_GEMM_TILE_N=128).
+    const char* env = std::getenv("SVDQ_GEMM_TILE_N");
+    const bool force128 = env && std::strcmp(env, "128") == 0;
+    h->n256 = !(bad & 8u) && d->R <= 32 && !force128;
+    h->lr_row_bytes = svdq::gemm_n256_lr_row_bytes(d->R);
+  }
 #undef CREATE_CUDA
 
   svdq_status s;
@@ -298,6 +361,14 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
   if ((s = make_tmap(&h->tm_pu, h->pu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d->R, d->N, (uint64_t)d->R * 2, 64, 128)) !=
       SVDQ_OK)
     return fail(s);
+  if (h->n256) {
+    if ((s = make_tmap(&h->tm_b256, h->qw, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->Kp / 2, d->N, h->Kp / 2, 128, 256)) !=
+        SVDQ_OK)
+      return fail(s);
+    if ((s = make_tmap(&h->tm_pu_fold, h->pu_fold, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d->R, d->N, (uint64_t)d->R * 2,
+                       h->lr_row_bytes / 2, 256, lr_swizzle(h->lr_row_bytes))) != SVDQ_OK)
+      return fail(s);
+  }
   *out = h;
   return SVDQ_OK;
 }
@@ -398,14 +469,8 @@ svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, 
   if ((s = make_tmap(&g.tm_a, ws + w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->Kp / 2, M, h->Kp / 2, 128, 128)) !=
       SVDQ_OK)
     return s;
-  g.tm_b = h->tm_b;
-  if ((s = make_tmap(&g.tm_l, ws + w.lr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->R, M, (uint64_t)h->R * 2, 64, 128)) !=
-      SVDQ_OK)
-    return s;
-  g.tm_pu = h->tm_pu;
   g.sfa = ws + w.sfa;
   g.sfb = h->sfb;
-  g.alpha = h->alpha;
   g.y = y;
   g.err = h->err;
   g.M = M;
@@ -413,6 +478,27 @@ svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, 
   g.R = h->R;
   g.k_tiles = h->k_tiles;
   g.ka_pad = h->ka_pad;
+  if (h->n256) {
+    g.tm_b = h->tm_b256;
+    if ((s = make_tmap(&g.tm_l, ws + w.lr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->R, M, (uint64_t)h->R * 2,
+                       h->lr_row_bytes / 2, 128, lr_swizzle(h->lr_row_bytes))) != SVDQ_OK)
+      return s;
+    g.tm_pu = h->tm_pu_fold;
+    g.alpha = h->alpha_fold;
+    g.y_tma = (h->N % 8) == 0;
+    if (g.y_tma &&
+        (s = make_tmap(&g.tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->N, M, (uint64_t)h->N * 2, 64, 32)) != SVDQ_OK)
+      return s;
+    cudaError_t e = svdq::launch_gemm_nvfp4_n256(g, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+    return SVDQ_OK;
+  }
+  g.tm_b = h->tm_b;
+  if ((s = make_tmap(&g.tm_l, ws + w.lr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->R, M, (uint64_t)h->R * 2, 64, 128)) !=
+      SVDQ_OK)
+    return s;
+  g.tm_pu = h->tm_pu;
+  g.alpha = h->alpha;
   cudaError_t e = svdq::launch_gemm_nvfp4_lr(g, stream);
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return SVDQ_OK;

@@ -42,11 +42,25 @@ struct GemmLaunch {
   const uint8_t* sfb;       // weight scale tiles
   const float* alpha;       // (N padded to 128) wcscales * wtscale
   void* y;                  // bf16 (M, N)
+  CUtensorMap tm_y;         // 128 x 256 GEMM, N % 8 == 0: y bf16 (M, N), box {64, 32}, 128B swizzle (TMA store)
+  bool y_tma;               // tm_y is valid
   unsigned* err;
   int M, N, R;
   int k_tiles;              // Kp rounded up to 256, divided by 256
   int ka_pad;               // K atoms per 128-row scale tile (= 4 * k_tiles)
 };
 cudaError_t launch_gemm_nvfp4_lr(const GemmLaunch& p, cudaStream_t stream);
+
+// The same product on 128 x 256 output tiles, with alpha folded into proj_up
+// (y = alpha' * (acc + L proj_up'^T)); the GemmLaunch fields then hold:
+//   tm_b   weight codes: box {128, 256}
+//   tm_l   L: box {lr_row_bytes / 2, 128}, swizzle of lr_row_bytes (32 or 64)
+//   tm_pu  proj_up' = bf16(proj_up / alpha) (N, R): box {lr_row_bytes / 2, 256}, same swizzle
+//   sfb    weight scale tiles, an even number of 128-row tiles
+//   alpha  alpha' (alpha, or 1 where alpha is 0)
+//   tm_y / y_tma  y through a shared-memory staging tile and TMA stores (N % 8 == 0)
+// Requires R <= 32 (the L / proj_up' tile must fit beside the ring and staging).
+int gemm_n256_lr_row_bytes(int R);
+cudaError_t launch_gemm_nvfp4_n256(const GemmLaunch& p, cudaStream_t stream);
 
 }  // namespace svdq

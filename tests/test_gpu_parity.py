@@ -100,8 +100,8 @@ def check_forward(layer, ck, rows=None):
 
 def check_forward_workspace(layer, ck):
     """White-box check of the forward path's quantizer output: the codes and
-    every replica of every tensor-core scale atom in the workspace must equal
-    the oracle's bytes (and the K padding must be zero)."""
+    every tensor-core scale atom in the workspace must equal the oracle's
+    bytes (and the K padding must be zero)."""
     M, K = ck.M, ck.K
     x = dev_bf16(ck.x)
     ws = layer.workspace(M)
@@ -116,14 +116,13 @@ def check_forward_workspace(layer, ck):
     np.testing.assert_array_equal(codes[:, : K // 2], c_ref)
     assert not codes[:, K // 2:].any()
     sfa = (M * Kp // 2 + 255) // 256 * 256
-    # [row tile][K atom][replica][row % 32][(row % 128) // 32][block in atom]
-    atoms = w[sfa: sfa + mtiles * ka_pad * 2048].reshape(mtiles, ka_pad, 4, 32, 4, 4)
+    # [row tile][K atom][row % 32][(row % 128) // 32][block in atom]
+    atoms = w[sfa: sfa + mtiles * ka_pad * 512].reshape(mtiles, ka_pad, 32, 4, 4)
     m = np.arange(M)
-    for r in range(4):
-        # (M, ka_pad, 4) -> (M, ka_pad * 4) scale bytes per 16-element block
-        rows = atoms[m // 128, :, r, m % 32, (m % 128) // 32, :].reshape(M, ka_pad * 4)
-        np.testing.assert_array_equal(rows[:, : K // 16], s_ref)
-        assert not rows[:, K // 16:].any()
+    # (M, ka_pad, 4) -> (M, ka_pad * 4) scale bytes per 16-element block
+    rows = atoms[m // 128, :, m % 32, (m % 128) // 32, :].reshape(M, ka_pad * 4)
+    np.testing.assert_array_equal(rows[:, : K // 16], s_ref)
+    assert not rows[:, K // 16:].any()
 
 
 # ------------------------------------------------------------------ number-format semantics
@@ -227,12 +226,44 @@ def test_full_workload_parity(name):
     (64, 2048, 640, 64, 128),
     (300, 4096, 128, 32, 0),    # split-K cluster reduction with ragged rows
 ])
-def test_ragged_shapes(M, K, N, R, rot):
+@pytest.mark.parametrize("tile", ["auto", "128"])
+def test_ragged_shapes(M, K, N, R, rot, tile, monkeypatch):
+    """Both GEMM kernels: "auto" takes the 128 x 256 tiles with alpha folded
+    into proj_up where R <= 64, "128" forces the 128 x 128 kernel."""
+    if tile == "128":
+        monkeypatch.setenv("SVDQ_GEMM_TILE_N", "128")
     ck = synthetic.make_checkpoint(M, K, N, R, seed=M + K + N + R, rotate_block=rot, dense_weight=bool(rot),
                                    wcscales="uniform", wtscale=0.75, name=f"ragged_{M}x{K}x{N}_r{R}_rot{rot}")
     layer = make_layer(ck)
     check_quantizer(layer, ck)
     check_forward_workspace(layer, ck)
+    check_forward(layer, ck)
+
+
+@pytest.mark.parametrize("tile", ["auto", "128"])
+def test_zero_alpha_columns(tile, monkeypatch):
+    """Columns with wcscales = 0 reduce to the rank-R branch alone, in both
+    GEMM kernels (the folded one gives them alpha' = 1 and zero weight scales)."""
+    if tile == "128":
+        monkeypatch.setenv("SVDQ_GEMM_TILE_N", "128")
+    ck = synthetic.make_checkpoint(150, 512, 520, 32, seed=12, wcscales="uniform",
+                                   name="zero_alpha_150x512x520_r32")
+    zero_cols = np.array([0, 1, 127, 128, 255, 256, 300, 511, 512, 519])
+    ck.wcscales = ck.wcscales.copy()
+    ck.wcscales[zero_cols] = 0
+    layer = make_layer(ck)
+    y = host_bf16_to_f64(check_forward(layer, ck))
+    xh = O.smooth_and_rotate(ck.x, ck.smooth_factor, 0)
+    lr = O.lowrank_down(xh, ck.proj_down) @ O.bf16_to_f32(ck.proj_up).astype(np.float64).T
+    assert_y_close(y[:, zero_cols], lr[:, zero_cols], "zero-alpha columns")
+
+
+def test_unfoldable_alpha_takes_plain_epilogue():
+    """wtscale = 2^-30 is outside the range where proj_up / alpha keeps bf16
+    precision, so the layer keeps alpha in the epilogue; results still match."""
+    ck = synthetic.make_checkpoint(140, 512, 384, 32, seed=13, wcscales="uniform", wtscale=2.0 ** -30,
+                                   name="tiny_alpha_140x512x384_r32")
+    layer = make_layer(ck)
     check_forward(layer, ck)
 
 
