@@ -14,19 +14,25 @@
 //
 // Persistent kernel, one CTA per SM, static tile schedule (M-tile fastest):
 //   warp 0 lane 0   TMA producer: per K step (256 FP4 elements) the activation
-//                   tile (128 rows) and weight tile (256 rows) of codes and
-//                   their compact scale atoms into a 3-deep ring; per tile the
-//                   L and proj_up' tiles.
+//                   tile (128 rows x 128 bytes) and weight tile (256 rows x 128
+//                   bytes), 128-byte swizzled, and their compact scale atoms
+//                   into a 3-deep ring; per tile the L and proj_up' tiles.
+//                   (Rows of 128 bytes: the TMA engine's throughput is set by
+//                   the rows it fetches more than by their bytes.)
 //   warp 1          owns 512 TMEM columns: accumulator [0,256), scale factors
-//                   [256,400) (three buffers of 48 columns: A in +0..15, B in
-//                   +16..47, 8 columns per K atom: rows 0-127 then 128-255).
+//                   [256,400) (three buffers of 48 columns: A atoms in +0..15,
+//                   B atom kb in +16+8kb .. +23+8kb, rows 0-127 then 128-255).
 //                   Lane 0 issues four MMAs per K step (M=128, N=256, K=64,
 //                   UE4M3 per 16), then the bf16 MMAs L . proj_up'^T (K = R)
 //                   into the same accumulator.
-//   warps 2-5       epilogue: TMEM -> registers, alpha' * acc -> bf16 into a
-//                   128B-swizzled staging tile (conflict-free), TMA stores to y.
-//   warps 6-9       scale warps: tcgen05.st of each stage's scale factors into
+//   warps 2-5       scale warps: tcgen05.st of each stage's scale factors into
 //                   their own 32-lane TMEM sub-partition (off the tensor pipe).
+//   warps 6-9       epilogue, one warp per 32-lane sub-partition: TMEM ->
+//                   registers, alpha' * acc -> bf16 into a swizzled
+//                   shared-memory box (conflict-free), read back row-major and
+//                   stored to y as full 128-byte row segments.
+// The accumulator is single-buffered, so the epilogue's drain is on the
+// critical path (two warps per sub-partition measured no faster).
 // Every wait is bounded; on expiry the CTA records an error, drains what it
 // started, frees TMEM and exits.
 #include <cuda_runtime.h>
@@ -40,17 +46,19 @@ namespace {
 constexpr int BM = 128, BN = 256;
 constexpr int kKTileBytes = 128;                 // 256 FP4 elements per row per stage
 constexpr int kStages = 3;
+constexpr int kAtoms = 4;                        // 64-element scale atoms per stage
 constexpr int kABytes = BM * kKTileBytes;        // 16 KB
 constexpr int kBBytes = BN * kKTileBytes;        // 32 KB
-constexpr int kSfaBytes = 4 * kSfAtomBytes;      // 4 K atoms, 128 rows (2 KB)
-constexpr int kSfbBytes = 2 * 4 * kSfAtomBytes;  // two 128-row halves (4 KB)
+constexpr int kSfaBytes = kAtoms * kSfAtomBytes;      // 128 rows (2 KB)
+constexpr int kSfbBytes = 2 * kAtoms * kSfAtomBytes;  // two 128-row halves (4 KB)
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;   // 54 KB
-constexpr int kThreads = 320;
-constexpr int kEpiWarps = 4;
-constexpr int kSfWarp0 = 6, kSfWarps = 4;
-constexpr int kSfBufs = kStages;                // the scale warps' buffer reuse needs kStages >= kSfBufs
+constexpr int kSfWarp0 = 2, kSfWarps = 4;
+constexpr int kEpiWarp0 = 6, kEpiWarps = 4;       // 4 or 8 (one or two per 32-lane sub-partition)
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
+constexpr int kSfBufs = kStages;                 // the scale warps' buffer reuse needs kStages >= kSfBufs
 constexpr int kSfCols = 48;
-constexpr int kStageOutBytes = 2 * 32 * 128;     // per epilogue warp: 32 rows x 128 columns bf16, two 64-column boxes
+constexpr int kEpiCols = BN * 4 / kEpiWarps;     // columns per epilogue warp
+constexpr int kStageOutBytes = 32 * 128;         // per epilogue warp: a 64-column x 32-row bf16 box
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColAcc = 0, kColSf = 256;
 
@@ -60,14 +68,14 @@ struct GParams {
   const float* alpha;     // alpha' (folded)
   __nv_bfloat16* y;
   unsigned* err;
-  int M, N, R, k_tiles, ka_pad;
+  int M, N, R, k_tiles, ka_pad;   // k_tiles: K steps of 256 elements
   int m_tiles, n_tiles;   // n_tiles of 256 columns
   int lr_row_bytes;       // bytes per row of the L / proj_up' tiles in shared memory (32 or 64)
-  int y_tma;              // write y through the staging tile and TMA stores
+  int y_vec;              // N % 8 == 0: y rows are 16-byte aligned, stored through the staging box
 };
 
-// Shared-memory descriptor for a K-major bf16 tile with 32/64/128-byte rows
-// (the matching swizzle), 8-row groups 8 * row_bytes apart.
+// Shared-memory descriptor for a K-major tile with 32/64/128-byte rows (the
+// matching swizzle), 8-row groups 8 * row_bytes apart.
 __device__ __forceinline__ uint64_t sdesc_kmajor_rows(uint32_t saddr, int row_bytes) {
   const uint64_t layout = row_bytes == 128 ? 2ull : (row_bytes == 64 ? 4ull : 6ull);
   return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(16u >> 4) << 16) |
@@ -77,13 +85,14 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_rows(uint32_t saddr, int row_by
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nvfp4_n256_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                            const __grid_constant__ CUtensorMap tm_l, const __grid_constant__ CUtensorMap tm_pu,
-                           const __grid_constant__ CUtensorMap tm_y, const GParams p) {
+                           const GParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int lr_l_bytes = BM * p.lr_row_bytes, lr_buf_bytes = (BM + BN) * p.lr_row_bytes;
   uint8_t* stages = base;
   uint8_t* OUT = stages + kStages * kStageBytes;                // kEpiWarps x kStageOutBytes
-  uint8_t* LRB = OUT + kEpiWarps * kStageOutBytes;              // one {L tile, proj_up' tile}
+  uint8_t* ALPHA = OUT + kEpiWarps * kStageOutBytes;            // kEpiWarps x kEpiCols floats
+  uint8_t* LRB = ALPHA + kEpiWarps * kEpiCols * 4;              // one {L tile, proj_up' tile}
   uint64_t* bars = reinterpret_cast<uint64_t*>(LRB + lr_buf_bytes);
   uint64_t* full = bars;                        // [kStages] TMA landed
   uint64_t* empty = full + kStages;             // [kStages] MMAs done reading the stage
@@ -147,11 +156,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(smem_u32(st), &tm_a, fb, kt * kKTileBytes, m0);
           tma_load_2d(smem_u32(st + kABytes), &tm_b, fb, kt * kKTileBytes, n0);
           bulk_load(smem_u32(st + kABytes + kBBytes),
-                    p.sfa + ((size_t)mt * p.ka_pad + (size_t)kt * 4) * kSfAtomBytes, kSfaBytes, fb);
+                    p.sfa + ((size_t)mt * p.ka_pad + (size_t)kt * kAtoms) * kSfAtomBytes, kSfaBytes, fb);
 #pragma unroll
           for (int h = 0; h < 2; ++h)
             bulk_load(smem_u32(st + kABytes + kBBytes + kSfaBytes + h * (kSfbBytes / 2)),
-                      p.sfb + ((size_t)(2 * nt + h) * p.ka_pad + (size_t)kt * 4) * kSfAtomBytes, kSfbBytes / 2, fb);
+                      p.sfb + ((size_t)(2 * nt + h) * p.ka_pad + (size_t)kt * kAtoms) * kSfAtomBytes, kSfbBytes / 2, fb);
           issued = g + 1;
           if (kt == p.k_tiles - 1) {
             // L / proj_up' tile of this output tile, read after its K loop;
@@ -195,9 +204,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t st = smem_u32(stages + s * kStageBytes);
           const uint32_t sf = tmem + kColSf + (uint32_t)b * kSfCols;
 #pragma unroll
-          for (int kb = 0; kb < 4; ++kb)
-            mma_nvfp4(tmem + kColAcc, sdesc_kmajor_sw128(st + kb * 32), sdesc_kmajor_sw128(st + kABytes + kb * 32),
-                      idesc_main, sf + 4 * kb, sf + 16 + 8 * kb, (kt | kb) != 0);
+          for (int kb = 0; kb < kAtoms; ++kb)
+            mma_nvfp4(tmem + kColAcc, sdesc_kmajor_rows(st + kb * 32, kKTileBytes),
+                      sdesc_kmajor_rows(st + kABytes + kb * 32, kKTileBytes), idesc_main, sf + 4 * kb,
+                      sf + 16 + 8 * kb, (kt | kb) != 0);
           tc_commit(smem_u32(&empty[s]));
         }
         if (!ok) break;
@@ -217,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= kSfWarp0) {
+  } else if (warp < kSfWarp0 + kSfWarps) {
     // Scale warps: stage g's scale atoms -> TMEM buffer g % kSfBufs of this
     // warp's lane quadrant.  Lane l's 16 bytes of an atom are the four columns
     // (rows l, l+32, l+64, l+96) of its TMEM lane.
@@ -228,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kt = 0; kt < p.k_tiles; ++kt, ++g) {
         const int s = g % kStages, b = g % kSfBufs;
         // Buffer b was last read by the MMAs of stage g - kSfBufs.  The whole
-        // warp agrees on the outcome before the warp-wide TMEM stores.
+        // warp agrees on the outcome before the warp-wide TMEM store.
         bool w = true;
         if (g >= kSfBufs)
           w = wait_bounded(smem_u32(&empty[(g - kSfBufs) % kStages]), ((g - kSfBufs) / kStages) & 1, abort_flag,
@@ -240,37 +250,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after_sync();
         const uint32_t sfs = smem_u32(stages + s * kStageBytes + kABytes + kBBytes) + lane * 16;
-        uint32_t va[32], vb[16];
+        // columns: A atom a -> 4a .. 4a+3; B atom kb -> 16+8kb+0..3 (rows 0-127), +4..7 (rows 128-255)
+        uint32_t v0[32], v1[16];            // columns 0..31 and 32..47 of the buffer
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {      // A atoms -> columns 4a .. 4a+3
-          const uint4 q = ld_shared_v4(sfs + a * kSfAtomBytes);
-          va[4 * a + 0] = q.x;
-          va[4 * a + 1] = q.y;
-          va[4 * a + 2] = q.z;
-          va[4 * a + 3] = q.w;
-        }
-#pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {   // B atom kb: rows 0-127 -> 16+8kb+0..3, rows 128-255 -> +4..7
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint4 q = ld_shared_v4(sfs + kSfaBytes + h * (kSfbBytes / 2) + kb * kSfAtomBytes);
-            const int c = 16 + 8 * kb + 4 * h;   // column in the buffer (a compile-time constant)
-            if (c < 32) {
-              va[c] = q.x;
-              va[c + 1] = q.y;
-              va[c + 2] = q.z;
-              va[c + 3] = q.w;
-            } else {
-              vb[c - 32] = q.x;
-              vb[c - 31] = q.y;
-              vb[c - 30] = q.z;
-              vb[c - 29] = q.w;
-            }
+        for (int i = 0; i < 12; ++i) {
+          // i = 0..3: A atoms; i = 4..11: B atom (i-4)>>1, half (i-4)&1
+          const uint32_t src = i < 4 ? sfs + i * kSfAtomBytes
+                                     : sfs + kSfaBytes + ((i - 4) & 1) * (kSfbBytes / 2) + ((i - 4) >> 1) * kSfAtomBytes;
+          const uint4 q = ld_shared_v4(src);
+          if (i < 8) {
+            v0[4 * i + 0] = q.x;
+            v0[4 * i + 1] = q.y;
+            v0[4 * i + 2] = q.z;
+            v0[4 * i + 3] = q.w;
+          } else {
+            v1[4 * i - 32] = q.x;
+            v1[4 * i - 31] = q.y;
+            v1[4 * i - 30] = q.z;
+            v1[4 * i - 29] = q.w;
           }
         }
-        const uint32_t col = lane_base + kColSf + (uint32_t)b * kSfCols;
-        tmem_st32(col, va);
-        tmem_st16(col + 32, vb);
+        tmem_st32(lane_base + kColSf + (uint32_t)b * kSfCols, v0);
+        tmem_st16(lane_base + kColSf + (uint32_t)b * kSfCols + 32, v1);
         tmem_st_wait();
         tc_fence_before_sync();
         __syncwarp();
@@ -278,82 +279,93 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // Epilogue: warps 2..5 cover TMEM lane quadrants 2, 3, 0, 1 (rows 32q..32q+31).
-    const int q = warp & 3;
+    // Epilogue warp e = warp - 6: TMEM lane quadrant q = warp & 3 (rows
+    // 32q..32q+31 of the tile), columns kEpiCols hc .. kEpiCols (hc + 1) - 1.
+    const int e = warp - kEpiWarp0;
+    const int q = warp & 3, hc = e >> 2;
     const int row = q * 32 + lane;
-    uint8_t* out = OUT + (warp - 2) * kStageOutBytes;
-    const uint32_t out_s = smem_u32(out);
-    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + kColAcc;
+    uint8_t* outp = OUT + e * kStageOutBytes;
+    float* alpha_w = reinterpret_cast<float*>(ALPHA + e * kEpiCols * 4);   // alpha'[n0 + 128hc ..] of this tile
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + kColAcc + (uint32_t)(hc * kEpiCols);
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
-      const int m0 = mt * BM, n0 = nt * BN, m = m0 + row;
+      const int m0 = mt * BM, m = m0 + row;
+      const int nw = nt * BN + hc * kEpiCols;     // first column of this warp's part of the tile
+      // alpha' of this tile into shared memory while the tensor core works on
+      // it (alpha' is padded to a multiple of 256 columns).
+      {
+        float4 a[kEpiCols / 128];
+#pragma unroll
+        for (int i = 0; i < kEpiCols / 128; ++i) a[i] = __ldg(reinterpret_cast<const float4*>(p.alpha + nw) + 32 * i + lane);
+        __syncwarp();                                   // every lane is done with the previous tile's copy
+#pragma unroll
+        for (int i = 0; i < kEpiCols / 128; ++i) reinterpret_cast<float4*>(alpha_w)[32 * i + lane] = a[i];
+        __syncwarp();
+      }
       const bool w = wait_bounded(smem_u32(acc_full), it & 1, abort_flag, p.err, kErrGemmTimeout);
       if (!__all_sync(0xffffffffu, w)) break;
       tc_fence_after_sync();
+      // 64-column chunks, each through the warp's staging box.
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        if (p.y_tma) {
-          // The staging tile was last read by the previous half's TMA stores.
-          if (lane == 0) bulk_wait_read<0>();
+      for (int pc = 0; pc < kEpiCols / 64; ++pc) {
+        const int nl0 = 64 * pc;                       // first column of the chunk in this warp's part
+        uint32_t acc[2][32];
+        tmem_ld32(lane_base + nl0, acc[0]);
+        tmem_ld32(lane_base + nl0 + 32, acc[1]);
+        tmem_ld_wait();
+        if (pc == kEpiCols / 64 - 1) {
+          // This warp has read its part of the accumulator.
+          tc_fence_before_sync();
           __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(acc_free));
         }
-#pragma unroll 1
-        for (int j = 0; j < 4; ++j) {
-          const int nl = 128 * h + 32 * j;            // first column of this chunk in the tile
-          uint32_t acc[32];
-          tmem_ld32(lane_base + nl, acc);
-          tmem_ld_wait();
-          if (h == 1 && j == 3) {
-            // The whole accumulator has been read: the next tile may start.
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(acc_free));
-          }
-          const float4* al = reinterpret_cast<const float4*>(p.alpha + n0 + nl);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int nl = nl0 + 32 * u;
           uint32_t o[16];
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const float4 a4 = __ldg(al + c);
-            o[2 * c] = pack_bf16x2(a4.x * __uint_as_float(acc[4 * c + 0]), a4.y * __uint_as_float(acc[4 * c + 1]));
-            o[2 * c + 1] = pack_bf16x2(a4.z * __uint_as_float(acc[4 * c + 2]), a4.w * __uint_as_float(acc[4 * c + 3]));
+            const float4 a4 = reinterpret_cast<const float4*>(alpha_w)[(nl >> 2) + c];   // same address in every lane
+            o[2 * c] = pack_bf16x2(a4.x * __uint_as_float(acc[u][4 * c + 0]), a4.y * __uint_as_float(acc[u][4 * c + 1]));
+            o[2 * c + 1] =
+                pack_bf16x2(a4.z * __uint_as_float(acc[u][4 * c + 2]), a4.w * __uint_as_float(acc[u][4 * c + 3]));
           }
-          if (p.y_tma) {
-            // 128B-swizzled box (64 columns x 32 rows): 16-byte chunk c of row r
-            // at r * 128 + ((c ^ (r & 7)) * 16); this chunk is columns 32 (j & 1) ..
-            const uint32_t box = out_s + (uint32_t)(j >> 1) * 4096u + (uint32_t)lane * 128u;
+          if (p.y_vec) {
+            // Row `lane` of a 64-column x 32-row box, 16-byte chunk c at
+            // lane * 128 + ((c ^ (lane & 7)) * 16): conflict-free both when each
+            // lane writes its row and when 8 lanes read one row back.
+            uint4* rowp = reinterpret_cast<uint4*>(outp + lane * 128);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint32_t chunk = (uint32_t)((j & 1) * 4 + c) ^ (uint32_t)(lane & 7);
-              st_shared_v4(box + chunk * 16u, make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]));
-            }
+            for (int c = 0; c < 4; ++c)
+              rowp[(4 * u + c) ^ (lane & 7)] = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
           } else if (m < p.M) {
-            __nv_bfloat16* dst = p.y + (size_t)m * p.N + n0 + nl;
+            __nv_bfloat16* dst = p.y + (size_t)m * p.N + nw + nl;
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-              if (n0 + nl + c < p.N) {
+              if (nw + nl + c < p.N) {
                 const uint32_t pr = o[c >> 1];
                 dst[c] = __ushort_as_bfloat16((unsigned short)((c & 1) ? (pr >> 16) : (pr & 0xFFFFu)));
               }
             }
           }
         }
-        if (p.y_tma) {
-          fence_proxy_async_smem();
+        if (p.y_vec) {
+          // Read the box back row-major (8 lanes x 16 bytes = one 128-byte row
+          // segment) and store it coalesced.
           __syncwarp();
-          if (lane == 0 && m0 + 32 * q < p.M) {
+          const int c = lane & 7, n = nw + nl0 + 8 * c;
 #pragma unroll
-            for (int bx = 0; bx < 2; ++bx) {
-              const int nc = n0 + 128 * h + 64 * bx;
-              if (nc < p.N) tma_store_2d(&tm_y, out_s + (uint32_t)bx * 4096u, nc, m0 + 32 * q);
-            }
-            bulk_commit();
+          for (int i = 0; i < 8; ++i) {
+            const int r = 4 * i + (lane >> 3);
+            const uint4 v = reinterpret_cast<const uint4*>(outp + r * 128)[c ^ (r & 7)];
+            const int mr = m0 + 32 * q + r;
+            if (mr < p.M && n < p.N) *reinterpret_cast<uint4*>(p.y + (size_t)mr * p.N + n) = v;
           }
+          __syncwarp();
         }
       }
     }
-    if (p.y_tma && lane == 0) bulk_wait<0>();
-    __syncwarp();
   }
 
   // ---- cleanup
@@ -385,7 +397,7 @@ cudaError_t launch_gemm_nvfp4_n256(const GemmLaunch& L, cudaStream_t stream) {
   if (L.M <= 0) return cudaSuccess;
   if (L.R > 32) return cudaErrorInvalidValue;
   const int row_bytes = gemm_n256_lr_row_bytes(L.R);
-  const size_t smem = 1024 + (size_t)kStages * kStageBytes + (size_t)kEpiWarps * kStageOutBytes +
+  const size_t smem = 1024 + (size_t)kStages * kStageBytes + (size_t)kEpiWarps * (kStageOutBytes + kEpiCols * 4) +
                       (size_t)(BM + BN) * row_bytes + 256;
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   cudaError_t e = ensure_smem_limit(gemm_nvfp4_n256_kernel, smem);
@@ -411,10 +423,10 @@ cudaError_t launch_gemm_nvfp4_n256(const GemmLaunch& L, cudaStream_t stream) {
   p.m_tiles = (L.M + BM - 1) / BM;
   p.n_tiles = (L.N + BN - 1) / BN;
   p.lr_row_bytes = row_bytes;
-  p.y_tma = L.y_tma ? 1 : 0;
+  p.y_vec = (L.N % 8) == 0;
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  gemm_nvfp4_n256_kernel<<<grid, kThreads, smem, stream>>>(L.tm_a, L.tm_b, L.tm_l, L.tm_pu, L.tm_y, p);
+  gemm_nvfp4_n256_kernel<<<grid, kThreads, smem, stream>>>(L.tm_a, L.tm_b, L.tm_l, L.tm_pu, p);
   return cudaGetLastError();
 }
 

@@ -34,6 +34,14 @@ __host__ __device__ __forceinline__ int sf_atom_offset(int r_in_tile, int j) {
   return (r_in_tile & 31) * 16 + (r_in_tile >> 5) * 4 + j;
 }
 
+// Slot of channel pair j in the smoothing-factor table: within each group of
+// 64 pairs (one 128-channel quantizer chunk) pair pp sits at (pp % 8) * 8 +
+// pp / 8, so the eight threads that read pairs 8t + i (t = 0..7) at once hit
+// eight consecutive 16-byte slots (no shared-memory bank conflict).
+__host__ __device__ __forceinline__ int lam_slot(int j) {
+  return (j & ~63) | ((j & 7) << 3) | ((j & 63) >> 3);
+}
+
 // Spin on an mbarrier phase.  Returns false, after setting *abort and the
 // error bit, when the wait exceeds kWaitTimeoutNs; returns false at once when
 // another thread of the CTA has already set *abort.

@@ -49,7 +49,7 @@ namespace {
 
 constexpr int kChunk = 128;                        // K elements per pipeline stage
 constexpr int kRows = 128;                         // token rows per CTA (TMEM lanes)
-constexpr int kStages = 2;
+constexpr int kMaxStages = 4;                     // ring depth: as many as shared memory allows
 constexpr int kXStageBytes = kRows * kChunk * 2;   // 32 KB: two 64-wide swizzled boxes
 constexpr int kXBoxBytes = kXStageBytes / 2;       // 16 KB
 constexpr int kLamStageBytes = kChunk * 8;         // float4 {-s0,-s1,1/s0,1/s1} per channel pair
@@ -71,6 +71,7 @@ struct QParams {
   int M, K, Kp, R;
   int codes_pitch, scales_pitch, k_limit, ka_pad;
   int chunks_per_cta, n_chunks, ksplit;
+  int stages;
 };
 
 // ---------------------------------------------------------------- packed fp32 helpers
@@ -166,16 +167,16 @@ __device__ __forceinline__ uint32_t quant_block(const uint64_t (&v)[8], float am
   const float q0 = amax * y6;
   const float q1 = fmaf(fmaf(q0, -6.0f, amax), y6, q0);
   const uint32_t sb = cvt_e4m3(q1);
-  w0 = w1 = 0u;
-  if (sb != 0u) {
-    const float2 sr = srec[sb];
-    const uint64_t ns = pk2(sr.x, sr.x), ys = pk2(sr.y, sr.y);
-    uint64_t q[8];
+  // Branch-free: a zero scale (table entry {+-0, 0}) divides every value to a
+  // finite +-0, and the mask then clears those codes to 0.
+  const float2 sr = srec[sb];
+  const uint64_t ns = pk2(sr.x, sr.x), ys = pk2(sr.y, sr.y);
+  uint64_t q[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) q[i] = NEG ? div_mk2(v[i], ns, ys) : div_rn2(v[i], ns, ys);
-    w0 = cvt_e2m1x8(lo2(q[0]), hi2(q[0]), lo2(q[1]), hi2(q[1]), lo2(q[2]), hi2(q[2]), lo2(q[3]), hi2(q[3]));
-    w1 = cvt_e2m1x8(lo2(q[4]), hi2(q[4]), lo2(q[5]), hi2(q[5]), lo2(q[6]), hi2(q[6]), lo2(q[7]), hi2(q[7]));
-  }
+  for (int i = 0; i < 8; ++i) q[i] = NEG ? div_mk2(v[i], ns, ys) : div_rn2(v[i], ns, ys);
+  const uint32_t keep = sb != 0u ? 0xFFFFFFFFu : 0u;
+  w0 = keep & cvt_e2m1x8(lo2(q[0]), hi2(q[0]), lo2(q[1]), hi2(q[1]), lo2(q[2]), hi2(q[2]), lo2(q[3]), hi2(q[3]));
+  w1 = keep & cvt_e2m1x8(lo2(q[4]), hi2(q[4]), lo2(q[5]), hi2(q[5]), lo2(q[6]), hi2(q[6]), lo2(q[7]), hi2(q[7]));
   return sb;
 }
 
@@ -264,7 +265,7 @@ __device__ __forceinline__ void store_scales(const QParams& p, int m, int row, i
 // to the tensor core.
 __device__ __forceinline__ void rotate_half(uint8_t* xs, const float4* lam4, const float2* srec, float y6, int row,
                                             int q, uint32_t (&cw)[8], uint32_t& sbytes) {
-  const float4* lam = lam4 + 32 * q;          // the 32 channel pairs of this half
+  // The 32 channel pairs of this half: pair 32q + 4c + i at lam_slot(32q + 4c + i).
   sbytes = 0;
   // The row's 128-element rotation block is split over lanes 2r (first 64)
   // and 2r+1 (last 64) of one warp.  Element e of this half is lane (e & 1)
@@ -277,7 +278,7 @@ __device__ __forceinline__ void rotate_half(uint8_t* xs, const float4* lam4, con
     const uint32_t xin[4] = {pw.x, pw.y, pw.z, pw.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float4 l = lam[4 * c + i];
+      const float4 l = lam4[lam_slot(32 * q + 4 * c + i)];
       v[4 * c + i] = div_rn2(bf16x2_to_f2(xin[i]), pk2(l.x, l.y), pk2(l.z, l.w));
       big = amax_nan(amax_nan(big, lo2(v[4 * c + i])), hi2(v[4 * c + i]));
     }
@@ -289,7 +290,7 @@ __device__ __forceinline__ void rotate_half(uint8_t* xs, const float4* lam4, con
       const uint32_t xin[4] = {pw.x, pw.y, pw.z, pw.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float4 l = lam[4 * c + i];
+        const float4 l = lam4[lam_slot(32 * q + 4 * c + i)];
         v[4 * c + i] = pk2(__fdiv_rn(__uint_as_float(xin[i] << 16), -l.x),
                            __fdiv_rn(__uint_as_float(xin[i] & 0xFFFF0000u), -l.y));
       }
@@ -357,40 +358,63 @@ __device__ __forceinline__ void smooth_cols(uint8_t* xs, const float4* lam4, con
   uint64_t nb[8], yb[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float4 l = lam4[8 * j + i];
+    const float4 l = lam4[8 * i + j];                 // pair 8j + i (see lam_slot)
     nb[i] = pk2(l.x, l.y);
     yb[i] = pk2(l.z, l.w);
   }
+  // All four rows are loaded before any is written back, and the common
+  // path has no per-row branch, so the four rows' dependency chains
+  // (divide, amax, scale, divide, convert) overlap.
+  uint32_t xin[4][8];
 #pragma unroll
   for (int rr = 0; rr < 4; ++rr) {
     const int row = r0 + 32 * rr;
     const uint4 p0 = *reinterpret_cast<const uint4*>(xs + xoff(row, 2 * j));
     const uint4 p1 = *reinterpret_cast<const uint4*>(xs + xoff(row, 2 * j + 1));
-    const uint32_t xin[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-    uint64_t v[8];
+    xin[rr][0] = p0.x; xin[rr][1] = p0.y; xin[rr][2] = p0.z; xin[rr][3] = p0.w;
+    xin[rr][4] = p1.x; xin[rr][5] = p1.y; xin[rr][6] = p1.z; xin[rr][7] = p1.w;
+  }
+  uint64_t v[4][8];
+  float amax[4];
+  bool finite = true;
+#pragma unroll
+  for (int rr = 0; rr < 4; ++rr) {
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      v[i] = NEG ? div_mk2(bf16x2_to_f2(xin[i]), nb[i], yb[i]) : div_rn2(bf16x2_to_f2(xin[i]), nb[i], yb[i]);
-    const float amax = amax8(v);
-    if (amax < 3.0e38f) {
-      sb[rr] = quant_block<NEG>(v, amax, srec, y6, cw[rr][0], cw[rr][1]);
-    } else {                           // overflow / NaN (rare): redo with the divide unit
+      v[rr][i] = NEG ? div_mk2(bf16x2_to_f2(xin[rr][i]), nb[i], yb[i]) : div_rn2(bf16x2_to_f2(xin[rr][i]), nb[i], yb[i]);
+    amax[rr] = amax8(v[rr]);
+    finite = finite && (amax[rr] < 3.0e38f);
+  }
+  if (finite) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float s0 = NEG ? lo2(nb[i]) : -lo2(nb[i]), s1 = NEG ? hi2(nb[i]) : -hi2(nb[i]);
-        v[i] = pk2(__fdiv_rn(__uint_as_float(xin[i] << 16), s0), __fdiv_rn(__uint_as_float(xin[i] & 0xFFFF0000u), s1));
-      }
-      sb[rr] = quant_block_slow(v, cw[rr][0], cw[rr][1]);
-      if (NEG) {
+    for (int rr = 0; rr < 4; ++rr) sb[rr] = quant_block<NEG>(v[rr], amax[rr], srec, y6, cw[rr][0], cw[rr][1]);
+  } else {
+    // A block holds +-inf or NaN (rare): such rows redo the divide with the
+    // divide unit and quantize on the IEEE path.  (Fully unrolled, so the
+    // per-row arrays stay in registers.)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] ^= 0x8000000080000000ull;   // write back -x_hat
+    for (int rr = 0; rr < 4; ++rr) {
+      if (amax[rr] < 3.0e38f) {
+        sb[rr] = quant_block<NEG>(v[rr], amax[rr], srec, y6, cw[rr][0], cw[rr][1]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float s0 = NEG ? lo2(nb[i]) : -lo2(nb[i]), s1 = NEG ? hi2(nb[i]) : -hi2(nb[i]);
+          v[rr][i] = pk2(__fdiv_rn(__uint_as_float(xin[rr][i] << 16), s0),
+                         __fdiv_rn(__uint_as_float(xin[rr][i] & 0xFFFF0000u), s1));
+        }
+        sb[rr] = quant_block_slow(v[rr], cw[rr][0], cw[rr][1]);
+        if (NEG) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[rr][i] ^= 0x8000000080000000ull;   // write back -x_hat
+        }
       }
     }
-    write_back_bf16(xs, row, 2 * j, v);
   }
+#pragma unroll
+  for (int rr = 0; rr < 4; ++rr) write_back_bf16(xs, r0 + 32 * rr, 2 * j, v[rr]);
 }
 
-// Stage the chunk's codes and compact scale atoms of the column mapping.
 __device__ __forceinline__ void stage_cols(uint8_t* cst, uint8_t* sst, int t, const uint32_t (&cw)[4][2],
                                            const uint32_t (&sb)[4]) {
   const int j = t & 7, r0 = t >> 3;
@@ -430,7 +454,7 @@ __device__ __forceinline__ void store_cols(const QParams& p, int m0, int t, int 
 }
 
 template <bool ROT, bool NEG, bool TILED>
-__global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
+__global__ void __launch_bounds__(kThreads, 1)
     quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_pdT,
                         const __grid_constant__ CUtensorMap tm_codes, const QParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -441,17 +465,17 @@ __global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
   const int R = p.R;
   const int pd_stage_bytes = R * kChunk * 2;     // two 64-wide boxes of R rows x 128 B
   uint8_t* X = base;
-  uint8_t* PD = X + kStages * kXStageBytes;
-  uint8_t* LAM = PD + kStages * pd_stage_bytes;
-  uint8_t* CST = LAM + kStages * kLamStageBytes;       // code staging, one per stage
-  uint8_t* SST = CST + kStages * kCodeStageBytes;      // scale-atom staging, one per stage
-  Tables* tabs = reinterpret_cast<Tables*>(SST + kStages * kSfStageBytes);
+  uint8_t* PD = X + p.stages * kXStageBytes;
+  uint8_t* LAM = PD + p.stages * pd_stage_bytes;
+  uint8_t* CST = LAM + p.stages * kLamStageBytes;       // code staging, one per stage
+  uint8_t* SST = CST + p.stages * kCodeStageBytes;      // scale-atom staging, one per stage
+  Tables* tabs = reinterpret_cast<Tables*>(SST + p.stages * kSfStageBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(tabs + 1);
   uint64_t* full = bars;                    // TMA landed
-  uint64_t* xready = bars + kStages;        // x_hat written back (256 arrivals)
-  uint64_t* empty = bars + 2 * kStages;     // MMA finished reading the stage
-  uint64_t* done = bars + 3 * kStages;      // all MMAs of this CTA finished
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 1);
+  uint64_t* xready = bars + p.stages;        // x_hat written back (256 arrivals)
+  uint64_t* empty = bars + 2 * p.stages;     // MMA finished reading the stage
+  uint64_t* done = bars + 3 * p.stages;      // all MMAs of this CTA finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * p.stages + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -461,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
   const uint32_t tmem_cols = R <= 32 ? 32u : (R <= 64 ? 64u : 128u);
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < p.stages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&xready[s]), kComputeThreads);
       mbar_init(smem_u32(&empty[s]), 1);
@@ -493,9 +517,9 @@ __global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
   if (warp == kProducerWarp) {
     if (lane == 0) {
       for (int i = 0; i < nch; ++i) {
-        const int s = i % kStages;
-        if (i >= kStages &&
-            !wait_bounded(smem_u32(&empty[s]), ((i / kStages) - 1) & 1, abort_flag, p.err, kErrQuantTimeout))
+        const int s = i % p.stages;
+        if (i >= p.stages &&
+            !wait_bounded(smem_u32(&empty[s]), ((i / p.stages) - 1) & 1, abort_flag, p.err, kErrQuantTimeout))
           break;
         const int kc = (c_begin + i) * kChunk;
         const uint32_t fb = smem_u32(&full[s]);
@@ -515,8 +539,8 @@ __global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, (uint32_t)R);
       for (int i = 0; i < nch; ++i) {
-        const int s = i % kStages;
-        const uint32_t par = (i / kStages) & 1;
+        const int s = i % p.stages;
+        const uint32_t par = (i / p.stages) & 1;
         if (!wait_bounded(smem_u32(&full[s]), par, abort_flag, p.err, kErrQuantTimeout)) break;
         if (!wait_bounded(smem_u32(&xready[s]), par, abort_flag, p.err, kErrQuantTimeout)) break;
         tc_fence_after_sync();
@@ -540,8 +564,8 @@ __global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
     const float y6 = __frcp_rn(6.0f);
     const int row2 = tid >> 1, q = tid & 1;      // rotated mapping: two threads per row
     for (int i = 0; i < nch; ++i) {
-      const int s = i % kStages;
-      if (!wait_bounded(smem_u32(&full[s]), (i / kStages) & 1, abort_flag, p.err, kErrQuantTimeout)) break;
+      const int s = i % p.stages;
+      if (!wait_bounded(smem_u32(&full[s]), (i / p.stages) & 1, abort_flag, p.err, kErrQuantTimeout)) break;
       const int kc = (c_begin + i) * kChunk;
       uint8_t* xs = X + s * kXStageBytes;
       const float4* lam = reinterpret_cast<const float4*>(LAM + s * kLamStageBytes);
@@ -672,9 +696,9 @@ __global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
 
   // ---- cleanup: after an abort, wait (bounded) for the copies this CTA started.
   if (warp == kProducerWarp && lane == 0 && *abort_flag) {
-    for (int s = 0; s < kStages && s < issued; ++s) {
-      const int last = s + ((issued - 1 - s) / kStages) * kStages;
-      wait_for(smem_u32(&full[s]), (last / kStages) & 1, 100000000ull);
+    for (int s = 0; s < p.stages && s < issued; ++s) {
+      const int last = s + ((issued - 1 - s) / p.stages) * p.stages;
+      wait_for(smem_u32(&full[s]), (last / p.stages) & 1, 100000000ull);
     }
   }
   if (warp == kMmaWarp && lane == 0) wait_for(smem_u32(done), 0, kWaitTimeoutNs);
@@ -686,8 +710,8 @@ __global__ void __launch_bounds__(kThreads, ROT ? 1 : 2)
   }
 }
 
-size_t smem_bytes(int R) {
-  return 1024 + (size_t)kStages * (kXStageBytes + R * kChunk * 2 + kLamStageBytes + kCodeStageBytes + kSfStageBytes) +
+size_t smem_bytes(int R, int stages) {
+  return 1024 + (size_t)stages * (kXStageBytes + R * kChunk * 2 + kLamStageBytes + kCodeStageBytes + kSfStageBytes) +
          sizeof(Tables) + 256;
 }
 
@@ -695,7 +719,7 @@ template <bool ROT, bool NEG, bool TILED>
 cudaError_t launch_impl(const CUtensorMap& tm_x, const CUtensorMap& tm_pdT, const CUtensorMap& tm_codes,
                         const QParams& p, int row_tiles, int ksplit, cudaStream_t stream) {
   auto kern = quantize_act_kernel<ROT, NEG, TILED>;
-  const size_t smem = smem_bytes(p.R);
+  const size_t smem = smem_bytes(p.R, p.stages);
   cudaError_t e = ensure_smem_limit(kern, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -720,14 +744,19 @@ cudaError_t launch_quantize_act(const QuantLaunch& L, cudaStream_t stream) {
   const int n_chunks = L.Kp / kChunk;
   const int row_tiles = (L.M + kRows - 1) / kRows;
   const bool rot = L.rotate_block == 128;
-  // Split K over a cluster until the grid covers the GPU (148 SMs; two CTAs
-  // per SM without rotation, one with).  Every CTA keeps at least one chunk.
-  const int slots = (rot || L.R > 64) ? 148 : 2 * 148;
-  const int max_split = rot ? 4 : 8;
+  // Split K over a cluster (up to 8 CTAs) as far as one wave of one CTA per
+  // SM allows.  Every CTA keeps at least one chunk.
+  static int num_sms = 0;
+  if (num_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (num_sms <= 0) num_sms = 148;
+  }
   int ksplit = 1;
-  for (int cand = max_split; cand >= 2; cand >>= 1) {
+  for (int cand = 8; cand >= 2; cand >>= 1) {
     const int cpc = (n_chunks + cand - 1) / cand;
-    if (cand <= n_chunks && (cand - 1) * cpc < n_chunks && row_tiles * cand <= 2 * slots) {
+    if (cand <= n_chunks && (cand - 1) * cpc < n_chunks && row_tiles * cand <= num_sms) {
       ksplit = cand;
       break;
     }
@@ -757,6 +786,9 @@ cudaError_t launch_quantize_act(const QuantLaunch& L, cudaStream_t stream) {
   p.chunks_per_cta = cpc;
   p.n_chunks = n_chunks;
   p.ksplit = ksplit;
+  // Deepest ring (up to kMaxStages) that fits in shared memory.
+  p.stages = kMaxStages;
+  while (p.stages > 2 && smem_bytes(L.R, p.stages) > 227 * 1024) --p.stages;
 
   if (rot) {
     return L.tiled_scales ? launch_impl<true, false, true>(L.tm_x, L.tm_pdT, L.tm_codes, p, row_tiles, ksplit, stream)

@@ -125,7 +125,8 @@ __global__ void transpose_proj_down(const __nv_bfloat16* __restrict__ pd, __nv_b
 
 // Per channel pair (k, k+1): {-s_k, -s_k+1, RN(1/s_k), RN(1/s_k+1)} and its
 // negation, the operands of the quantizer's two-lane correctly rounded
-// division by s or by -s; padding channels get s = 1.  bad bit 2: a zero or
+// division by s or by -s; padding channels get s = 1.  Stored in the
+// quantizer's bank-conflict-free order (svdq::lam_slot).  bad bit 2: a zero or
 // non-finite factor; bit 4: a negative one.
 __global__ void prepare_smooth(const __nv_bfloat16* __restrict__ sf, float4* __restrict__ lam4,
                                float4* __restrict__ lam4_neg, int K, int Kp, unsigned* bad) {
@@ -138,8 +139,9 @@ __global__ void prepare_smooth(const __nv_bfloat16* __restrict__ sf, float4* __r
       if (l0 < 0.0f || l1 < 0.0f) atomicOr(bad, 4u);
     }
     const float r0 = __frcp_rn(l0), r1 = __frcp_rn(l1);
-    lam4[j] = make_float4(-l0, -l1, r0, r1);
-    lam4_neg[j] = make_float4(l0, l1, -r0, -r1);
+    const int o = svdq::lam_slot(j);
+    lam4[o] = make_float4(-l0, -l1, r0, r1);
+    lam4_neg[o] = make_float4(l0, l1, -r0, -r1);
   }
 }
 
@@ -485,10 +487,6 @@ svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, 
       return s;
     g.tm_pu = h->tm_pu_fold;
     g.alpha = h->alpha_fold;
-    g.y_tma = (h->N % 8) == 0;
-    if (g.y_tma &&
-        (s = make_tmap(&g.tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->N, M, (uint64_t)h->N * 2, 64, 32)) != SVDQ_OK)
-      return s;
     cudaError_t e = svdq::launch_gemm_nvfp4_n256(g, stream);
     if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
     return SVDQ_OK;

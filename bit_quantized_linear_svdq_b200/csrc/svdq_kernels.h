@@ -42,8 +42,6 @@ struct GemmLaunch {
   const uint8_t* sfb;       // weight scale tiles
   const float* alpha;       // (N padded to 128) wcscales * wtscale
   void* y;                  // bf16 (M, N)
-  CUtensorMap tm_y;         // 128 x 256 GEMM, N % 8 == 0: y bf16 (M, N), box {64, 32}, 128B swizzle (TMA store)
-  bool y_tma;               // tm_y is valid
   unsigned* err;
   int M, N, R;
   int k_tiles;              // Kp rounded up to 256, divided by 256
@@ -58,7 +56,6 @@ cudaError_t launch_gemm_nvfp4_lr(const GemmLaunch& p, cudaStream_t stream);
 //   tm_pu  proj_up' = bf16(proj_up / alpha) (N, R): box {lr_row_bytes / 2, 256}, same swizzle
 //   sfb    weight scale tiles, an even number of 128-row tiles
 //   alpha  alpha' (alpha, or 1 where alpha is 0)
-//   tm_y / y_tma  y through a shared-memory staging tile and TMA stores (N % 8 == 0)
 // Requires R <= 32 (the L / proj_up' tile must fit beside the ring and staging).
 int gemm_n256_lr_row_bytes(int R);
 cudaError_t launch_gemm_nvfp4_n256(const GemmLaunch& p, cudaStream_t stream);
