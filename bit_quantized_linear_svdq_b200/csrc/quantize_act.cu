@@ -58,9 +58,21 @@ constexpr int kLamStageBytes = kChunk * 8;         // float4 {-s0,-s1,1/s0,1/s1}
 // chunk's two scale atoms, each to its four replicas).
 constexpr int kCodeStageBytes = kRows * kChunk / 2;   // 8 KB
 constexpr int kSfStageBytes = 2 * kSfAtomBytes;       // 1 KB
-constexpr int kComputeThreads = 256;
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
-constexpr int kThreads = 320;
+// Thread layout: 8 compute warps, then the TMA producer warp and the MMA
+// warp.  The unrotated path gives each thread four rows of one 16-channel
+// block column (measured faster than 16 warps of two rows, which need fewer
+// registers than the four-row chains want); the rotated path gives two
+// threads to each row.
+template <bool ROT>
+struct QCfg {
+  static constexpr int kComputeWarps = 8;
+  static constexpr int kComputeThreads = 32 * kComputeWarps;
+  static constexpr int kRowsPerThread = ROT ? 1 : 4;     // unrotated path: rows r0 + (128 / 4) * rr
+  static constexpr int kProducerWarp = kComputeWarps, kMmaWarp = kComputeWarps + 1;
+  static constexpr int kThreads = 32 * (kComputeWarps + 2);
+};
+constexpr int kColRowsPerThread = QCfg<false>::kRowsPerThread;
+constexpr int kColRowStride = kRows / kColRowsPerThread;   // 64
 
 struct QParams {
   const float4* lam4;
@@ -133,11 +145,21 @@ __device__ __forceinline__ float amax_nan(float acc, float v) {
   return r;
 }
 
+// NaN-propagating max of three magnitudes (sm_100 three-input form).
+__device__ __forceinline__ float amax3_nan(float a, float b, float c) {
+  float r;
+  asm("max.NaN.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// max |v| over a 16-element block (NaN if any element is NaN): eight
+// three-input maxes in a tree of depth three.
 __device__ __forceinline__ float amax8(const uint64_t (&v)[8]) {
-  float a = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) a = amax_nan(amax_nan(a, lo2(v[i])), hi2(v[i]));
-  return a;
+  const float m0 = amax3_nan(lo2(v[0]), hi2(v[0]), lo2(v[1]));
+  const float m1 = amax3_nan(hi2(v[1]), lo2(v[2]), hi2(v[2]));
+  const float m2 = amax3_nan(lo2(v[3]), hi2(v[3]), lo2(v[4]));
+  const float m3 = amax3_nan(hi2(v[4]), lo2(v[5]), hi2(v[5]));
+  const float m4 = amax3_nan(lo2(v[6]), hi2(v[6]), lo2(v[7]));
+  return amax3_nan(amax3_nan(m0, m1, m2), amax3_nan(m3, m4, hi2(v[7])), 0.0f);
 }
 
 // bf16 word (two channels) -> packed fp32 pair
@@ -353,7 +375,8 @@ __device__ __forceinline__ void rotate_half(uint8_t* xs, const float4* lam4, con
 // positive) over the sign-fixed one.
 template <bool NEG>
 __device__ __forceinline__ void smooth_cols(uint8_t* xs, const float4* lam4, const float2* srec, float y6, int t,
-                                            uint32_t (&cw)[4][2], uint32_t (&sb)[4]) {
+                                            uint32_t (&cw)[kColRowsPerThread][2], uint32_t (&sb)[kColRowsPerThread]) {
+  constexpr int RPT = kColRowsPerThread;
   const int j = t & 7, r0 = t >> 3;
   uint64_t nb[8], yb[8];
 #pragma unroll
@@ -362,23 +385,23 @@ __device__ __forceinline__ void smooth_cols(uint8_t* xs, const float4* lam4, con
     nb[i] = pk2(l.x, l.y);
     yb[i] = pk2(l.z, l.w);
   }
-  // All four rows are loaded before any is written back, and the common
-  // path has no per-row branch, so the four rows' dependency chains
+  // The thread's rows are all loaded before any is written back, and the
+  // common path has no per-row branch, so the rows' dependency chains
   // (divide, amax, scale, divide, convert) overlap.
-  uint32_t xin[4][8];
+  uint32_t xin[RPT][8];
 #pragma unroll
-  for (int rr = 0; rr < 4; ++rr) {
-    const int row = r0 + 32 * rr;
+  for (int rr = 0; rr < RPT; ++rr) {
+    const int row = r0 + kColRowStride * rr;
     const uint4 p0 = *reinterpret_cast<const uint4*>(xs + xoff(row, 2 * j));
     const uint4 p1 = *reinterpret_cast<const uint4*>(xs + xoff(row, 2 * j + 1));
     xin[rr][0] = p0.x; xin[rr][1] = p0.y; xin[rr][2] = p0.z; xin[rr][3] = p0.w;
     xin[rr][4] = p1.x; xin[rr][5] = p1.y; xin[rr][6] = p1.z; xin[rr][7] = p1.w;
   }
-  uint64_t v[4][8];
-  float amax[4];
+  uint64_t v[RPT][8];
+  float amax[RPT];
   bool finite = true;
 #pragma unroll
-  for (int rr = 0; rr < 4; ++rr) {
+  for (int rr = 0; rr < RPT; ++rr) {
 #pragma unroll
     for (int i = 0; i < 8; ++i)
       v[rr][i] = NEG ? div_mk2(bf16x2_to_f2(xin[rr][i]), nb[i], yb[i]) : div_rn2(bf16x2_to_f2(xin[rr][i]), nb[i], yb[i]);
@@ -387,13 +410,13 @@ __device__ __forceinline__ void smooth_cols(uint8_t* xs, const float4* lam4, con
   }
   if (finite) {
 #pragma unroll
-    for (int rr = 0; rr < 4; ++rr) sb[rr] = quant_block<NEG>(v[rr], amax[rr], srec, y6, cw[rr][0], cw[rr][1]);
+    for (int rr = 0; rr < RPT; ++rr) sb[rr] = quant_block<NEG>(v[rr], amax[rr], srec, y6, cw[rr][0], cw[rr][1]);
   } else {
     // A block holds +-inf or NaN (rare): such rows redo the divide with the
     // divide unit and quantize on the IEEE path.  (Fully unrolled, so the
     // per-row arrays stay in registers.)
 #pragma unroll
-    for (int rr = 0; rr < 4; ++rr) {
+    for (int rr = 0; rr < RPT; ++rr) {
       if (amax[rr] < 3.0e38f) {
         sb[rr] = quant_block<NEG>(v[rr], amax[rr], srec, y6, cw[rr][0], cw[rr][1]);
       } else {
@@ -412,15 +435,16 @@ __device__ __forceinline__ void smooth_cols(uint8_t* xs, const float4* lam4, con
     }
   }
 #pragma unroll
-  for (int rr = 0; rr < 4; ++rr) write_back_bf16(xs, r0 + 32 * rr, 2 * j, v[rr]);
+  for (int rr = 0; rr < RPT; ++rr) write_back_bf16(xs, r0 + kColRowStride * rr, 2 * j, v[rr]);
 }
 
-__device__ __forceinline__ void stage_cols(uint8_t* cst, uint8_t* sst, int t, const uint32_t (&cw)[4][2],
-                                           const uint32_t (&sb)[4]) {
+__device__ __forceinline__ void stage_cols(uint8_t* cst, uint8_t* sst, int t,
+                                           const uint32_t (&cw)[kColRowsPerThread][2],
+                                           const uint32_t (&sb)[kColRowsPerThread]) {
   const int j = t & 7, r0 = t >> 3;
 #pragma unroll
-  for (int rr = 0; rr < 4; ++rr) {
-    const int row = r0 + 32 * rr;
+  for (int rr = 0; rr < kColRowsPerThread; ++rr) {
+    const int row = r0 + kColRowStride * rr;
     *reinterpret_cast<uint2*>(cst + row * (kChunk / 2) + j * 8) = make_uint2(cw[rr][0], cw[rr][1]);
     sst[(j >> 2) * kSfAtomBytes + sf_atom_offset(row, j & 3)] = (uint8_t)sb[rr];
   }
@@ -436,14 +460,15 @@ __device__ __forceinline__ void stage_half(uint8_t* cst, uint8_t* sst, int row, 
 }
 
 template <bool TILED>
-__device__ __forceinline__ void store_cols(const QParams& p, int m0, int t, int kc, const uint32_t (&cw)[4][2],
-                                           const uint32_t (&sb)[4]) {
+__device__ __forceinline__ void store_cols(const QParams& p, int m0, int t, int kc,
+                                           const uint32_t (&cw)[kColRowsPerThread][2],
+                                           const uint32_t (&sb)[kColRowsPerThread]) {
   const int j = t & 7, r0 = t >> 3;
   const int k = kc + 16 * j;
   if (k >= p.k_limit) return;
 #pragma unroll
-  for (int rr = 0; rr < 4; ++rr) {
-    const int row = r0 + 32 * rr, m = m0 + row;
+  for (int rr = 0; rr < kColRowsPerThread; ++rr) {
+    const int row = r0 + kColRowStride * rr, m = m0 + row;
     if (m >= p.M) continue;
     *reinterpret_cast<uint2*>(p.codes + (size_t)m * p.codes_pitch + (k >> 1)) = make_uint2(cw[rr][0], cw[rr][1]);
     if (TILED) {
@@ -454,9 +479,11 @@ __device__ __forceinline__ void store_cols(const QParams& p, int m0, int t, int 
 }
 
 template <bool ROT, bool NEG, bool TILED>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(QCfg<ROT>::kThreads, 1)
     quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_pdT,
                         const __grid_constant__ CUtensorMap tm_codes, const QParams p) {
+  constexpr int kComputeThreads = QCfg<ROT>::kComputeThreads;
+  constexpr int kProducerWarp = QCfg<ROT>::kProducerWarp, kMmaWarp = QCfg<ROT>::kMmaWarp;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // Round up to 1024 bytes by pointer arithmetic on the __shared__ array, so
   // every access below stays a shared-memory access (an integer round trip
@@ -469,7 +496,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* LAM = PD + p.stages * pd_stage_bytes;
   uint8_t* CST = LAM + p.stages * kLamStageBytes;       // code staging, one per stage
   uint8_t* SST = CST + p.stages * kCodeStageBytes;      // scale-atom staging, one per stage
-  Tables* tabs = reinterpret_cast<Tables*>(SST + p.stages * kSfStageBytes);
+  float* recv = reinterpret_cast<float*>(SST + p.stages * kSfStageBytes);   // [ksplit][128/ksplit rows][R]: partial L
+  Tables* tabs = reinterpret_cast<Tables*>(reinterpret_cast<uint8_t*>(recv) + (size_t)kRows * R * 4);
   uint64_t* bars = reinterpret_cast<uint64_t*>(tabs + 1);
   uint64_t* full = bars;                    // TMA landed
   uint64_t* xready = bars + p.stages;        // x_hat written back (256 arrivals)
@@ -544,6 +572,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_bounded(smem_u32(&full[s]), par, abort_flag, p.err, kErrQuantTimeout)) break;
         if (!wait_bounded(smem_u32(&xready[s]), par, abort_flag, p.err, kErrQuantTimeout)) break;
         tc_fence_after_sync();
+        if (TILED) {
+          // Every compute thread has staged its codes and scales (xready):
+          // write the chunk's code tile and its two adjacent scale atoms.
+          const int kc = (c_begin + i) * kChunk;
+          tma_store_2d(&tm_codes, smem_u32(CST + s * kCodeStageBytes), kc / 2, m0);
+          bulk_store(p.scales + ((size_t)blockIdx.x * p.ka_pad + kc / 64) * kSfAtomBytes,
+                     smem_u32(SST + s * kSfStageBytes), kSfStageBytes);
+          bulk_commit();
+        }
         const uint32_t xa = smem_u32(X + s * kXStageBytes);
         const uint32_t pa = smem_u32(PD + s * pd_stage_bytes);
 #pragma unroll
@@ -552,15 +589,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = sdesc_kmajor_sw128(pa + (kk >> 2) * (R * 128) + (kk & 3) * 32);
           mma_bf16(tmem, ad, bd, idesc, (i | kk) != 0);
         }
+        // The stage (and its staging buffers) is released only once the stores
+        // have read the staging buffers.
+        if (TILED) bulk_wait_read<0>();
         tc_commit(smem_u32(&empty[s]));
       }
       // Arrives when every MMA issued above has finished; waited on below
       // before the tensor memory is released.
       tc_commit(smem_u32(done));
+      if (TILED) bulk_wait<0>();
     }
     __syncwarp();
   } else {
-    // warps 0-7: the chunk's 128 rows x 128 channels
+    // compute warps: the chunk's 128 rows x 128 channels
     const float y6 = __frcp_rn(6.0f);
     const int row2 = tid >> 1, q = tid & 1;      // rotated mapping: two threads per row
     for (int i = 0; i < nch; ++i) {
@@ -570,16 +611,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* xs = X + s * kXStageBytes;
       const float4* lam = reinterpret_cast<const float4*>(LAM + s * kLamStageBytes);
       uint32_t cw8[8], sbytes = 0;                 // rotated mapping
-      uint32_t cw[4][2], sb[4];                    // column mapping
+      uint32_t cw[kColRowsPerThread][2], sb[kColRowsPerThread];   // column mapping
       if (ROT)
         rotate_half(xs, lam, tabs->srec, y6, row2, q, cw8, sbytes);
       else
         smooth_cols<NEG>(xs, lam, tabs->srec, y6, tid, cw, sb);
       if (TILED) {
-        // The staging buffer of this stage was last read by the stores of
-        // chunk i - 2; tid 0 waits for them, the barrier tells everyone.
-        if (tid == 0) bulk_wait_read<1>();
-        named_bar(1, kComputeThreads);
+        // The stores that last read this stage's staging buffers finished
+        // before the stage was released for this chunk's load.
         uint8_t* cst = CST + s * kCodeStageBytes;
         uint8_t* sst = SST + s * kSfStageBytes;
         if (ROT)
@@ -589,26 +628,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();                    // x_hat (and staging) -> async proxy
       mbar_arrive(smem_u32(&xready[s]));
-      if (TILED) {
-        named_bar(1, kComputeThreads);
-        if (tid == 0) {
-          tma_store_2d(&tm_codes, smem_u32(CST + s * kCodeStageBytes), kc / 2, m0);
-          // the chunk's two scale atoms are adjacent in the tiled layout
-          bulk_store(p.scales + ((size_t)blockIdx.x * p.ka_pad + kc / 64) * kSfAtomBytes,
-                     smem_u32(SST + s * kSfStageBytes), kSfStageBytes);
-          bulk_commit();
-        }
-      } else if (ROT) {
+      if (!TILED && ROT) {
         const int m = m0 + row2, k0 = kc + 64 * q;
         if (m < p.M && k0 < p.k_limit) {
           store_codes<false>(p, m, k0, cw8);
           store_scales<false>(p, m, row2, k0, sbytes);
         }
-      } else {
+      } else if (!TILED) {
         store_cols<false>(p, m0, tid, kc, cw, sb);
       }
     }
-    if (TILED && tid == 0) bulk_wait<0>();
     // The CTA that owns the last chunk zero-fills the scale atoms beyond Kp
     // (the GEMM's last K tile reads them and they must be finite).
     if (TILED && tid < kRows && m0 + tid < p.M && c_begin + nch == p.n_chunks) {
@@ -620,14 +649,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---- rank-R down-projection: TMEM -> L (cluster reduction when K is split)
+  // With K split over a cluster, rank q owns rows [q * 128/ksplit, (q+1) *
+  // 128/ksplit) of the tile: every CTA pushes its partial sums of those rows
+  // into slot (its rank) of the owner's receive buffer with DSMEM stores,
+  // one cluster barrier publishes them, and each owner adds its slots in rank
+  // order (a fixed order: the result does not depend on timing).
   const bool want_lr = p.lowrank != nullptr;
-  const int pstride = R + 4;                          // padded row stride (floats) of the partial tile
-  float* partial = reinterpret_cast<float*>(base);   // reuses the x / proj_down ring once all MMAs are done
+  const int rows_per = kRows / p.ksplit;
   if (want_lr && tid < kRows) {
     // warps 0-3 read TMEM lane quadrants 0-3: thread tid owns row tid.
     const bool ok = wait_bounded(smem_u32(done), 0, abort_flag, p.err, kErrQuantTimeout);
     tc_fence_after_sync();
     const int row = tid, m = m0 + row;
+    const uint32_t owner = (uint32_t)(row / rows_per);
+    const uint32_t dst0 = p.ksplit > 1 ? mapa_shared(smem_u32(recv) + (uint32_t)(((int)cluster_ctarank() * rows_per +
+                                                                                  row % rows_per) * R * 4),
+                                                     owner)
+                                       : 0u;
     if (ok) {
       for (int j = 0; j < R; j += 16) {
         uint32_t r[16];
@@ -650,48 +688,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15])));
           }
         } else {
-          float4* dst = reinterpret_cast<float4*>(partial + row * pstride + j);
 #pragma unroll
           for (int t = 0; t < 4; ++t)
-            dst[t] = make_float4(__uint_as_float(r[4 * t]), __uint_as_float(r[4 * t + 1]),
-                                 __uint_as_float(r[4 * t + 2]), __uint_as_float(r[4 * t + 3]));
+            st_shared_cluster_v4(dst0 + (uint32_t)(j + 4 * t) * 4u, __uint_as_float(r[4 * t]),
+                                 __uint_as_float(r[4 * t + 1]), __uint_as_float(r[4 * t + 2]),
+                                 __uint_as_float(r[4 * t + 3]));
         }
       }
     }
   }
   if (want_lr && p.ksplit > 1) {
-    cluster_sync();
+    cluster_sync();                    // every partial has landed in its owner's buffer
     if (tid < kComputeThreads && !*abort_flag) {
-      // Rank r reduces rows [r * 128/ksplit, (r+1) * 128/ksplit) over all
-      // ranks (rank order fixed), four columns per step.
       const uint32_t rank = cluster_ctarank();
-      const int rows_per = kRows / p.ksplit;
       const int r4 = R / 4;
-      const uint32_t pbase = smem_u32(partial);
       for (int idx = tid; idx < rows_per * r4; idx += kComputeThreads) {
-        const int row = (int)rank * rows_per + idx / r4, col = 4 * (idx % r4);
-        const int m = m0 + row;
+        const int rl = idx / r4, col = 4 * (idx % r4);
+        const int m = m0 + (int)rank * rows_per + rl;
         if (m >= p.M) continue;
-        const uint32_t off = pbase + (uint32_t)((row * pstride + col) * 4);
-        float4 v[8];
-#pragma unroll
-        for (int qr = 0; qr < 8; ++qr)
-          if (qr < p.ksplit) v[qr] = ld_shared_cluster_v4(mapa_shared(off, (uint32_t)qr));
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-        for (int qr = 0; qr < 8; ++qr) {
-          if (qr < p.ksplit) {
-            a0 += v[qr].x;
-            a1 += v[qr].y;
-            a2 += v[qr].z;
-            a3 += v[qr].w;
-          }
+        for (int q = 0; q < p.ksplit; ++q) {
+          const float4 v = *reinterpret_cast<const float4*>(recv + (size_t)(q * rows_per + rl) * R + col);
+          a0 += v.x;
+          a1 += v.y;
+          a2 += v.z;
+          a3 += v.w;
         }
         *reinterpret_cast<uint2*>(p.lowrank + (size_t)m * R + col) =
             make_uint2(pack_bf16x2(a0, a1), pack_bf16x2(a2, a3));
       }
     }
-    cluster_sync();
   }
 
   // ---- cleanup: after an abort, wait (bounded) for the copies this CTA started.
@@ -712,6 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t smem_bytes(int R, int stages) {
   return 1024 + (size_t)stages * (kXStageBytes + R * kChunk * 2 + kLamStageBytes + kCodeStageBytes + kSfStageBytes) +
+         (size_t)kRows * R * 4 +
          sizeof(Tables) + 256;
 }
 
@@ -724,7 +751,7 @@ cudaError_t launch_impl(const CUtensorMap& tm_x, const CUtensorMap& tm_pdT, cons
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)row_tiles, (unsigned)ksplit, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(QCfg<ROT>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

@@ -161,6 +161,42 @@ def test_convert_semantics_ties_signed_zero_saturation():
     check_forward(layer2, ck)
 
 
+@pytest.mark.filterwarnings("ignore:overflow encountered:RuntimeWarning")   # x / lambda overflows to inf by design
+@pytest.mark.parametrize("neg_lambda", [False, True])
+def test_non_finite_blocks(neg_lambda):
+    """Blocks holding +-inf or NaN, or finite values that overflow once divided
+    by a small smoothing factor, take the IEEE path: a NaN block gets scale byte
+    0x7F and zero codes, an infinite amax saturates the scale to 448.  Codes and
+    scales are compared bit-exactly in the public and the tensor-core layouts;
+    every other block of the same rows must be unaffected."""
+    ck = synthetic.make_checkpoint(200, 512, 256, 32, seed=14, name="non_finite_200x512")
+    x = ck.x.copy()
+    bf = lambda f: np.array([f], dtype=np.float32).view(np.uint32)[0] >> 16
+    x[3, 5] = bf(np.inf)
+    x[3, 40] = bf(-np.inf)
+    x[77, 100] = bf(np.nan)
+    x[130, 16 * 9 + 3] = bf(np.nan)
+    x[130, 16 * 9 + 4] = bf(-np.inf)
+    x[199, 511] = bf(3.0e38)            # overflows after dividing by a factor < 1
+    x[150, 256:272] = bf(-3.0e38)
+    ck.x = x
+    sm = ck.smooth_factor.copy()
+    sm[511] = bf(0.25)
+    sm[256:272] = bf(0.5)
+    if neg_lambda:
+        sm[::7] = sm[::7] | 0x8000
+    ck.smooth_factor = sm
+    layer = make_layer(ck)
+    xd = dev_bf16(ck.x)
+    codes, scales, _ = layer.quantize_act(xd, with_lowrank=False)
+    torch.cuda.synchronize()
+    c_ref, s_ref, _ = O.quantize_act(ck.x, ck.smooth_factor, 0)
+    np.testing.assert_array_equal(scales.cpu().numpy(), s_ref)
+    np.testing.assert_array_equal(codes.cpu().numpy(), c_ref)
+    assert s_ref[77, 100 // 16] == 0x7F and s_ref[3, 0] == 0x7E     # the cases above really occur
+    check_forward_workspace(layer, ck)
+
+
 def test_negative_smooth_factors_random():
     ck = synthetic.make_checkpoint(150, 512, 256, 32, seed=12, name="negative_smooth")
     lam = O.bf16_to_f32(ck.smooth_factor).copy()
