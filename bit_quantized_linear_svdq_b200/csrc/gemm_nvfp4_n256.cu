@@ -122,6 +122,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  // Everything above overlaps the previous kernel's tail (programmatic
+  // dependent launch); nothing below runs before it has completed.
+  griddep_wait();
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
@@ -130,6 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  if (tid == 0) griddep_launch_dependents();
 
   int issued = 0, lr_issued = 0;
 
@@ -426,8 +430,17 @@ cudaError_t launch_gemm_nvfp4_n256(const GemmLaunch& L, cudaStream_t stream) {
   p.y_vec = (L.N % 8) == 0;
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  gemm_nvfp4_n256_kernel<<<grid, kThreads, smem, stream>>>(L.tm_a, L.tm_b, L.tm_l, L.tm_pu, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_n256_kernel, L.tm_a, L.tm_b, L.tm_l, L.tm_pu, p);
 }
 
 }  // namespace svdq

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cstdlib>
 #include <cuda_runtime.h>
 
 #include <map>
@@ -69,6 +70,18 @@ __device__ __forceinline__ bool wait_for(uint32_t bar, uint32_t parity, uint64_t
     if (globaltimer_ns() - t0 > timeout_ns) return false;
   }
   return true;
+}
+
+// Programmatic dependent launch of the hot-path kernels (on unless the
+// environment sets SVDQ_PDL=0): a kernel's launch and prologue overlap the
+// previous kernel's tail; each kernel waits (griddep_wait) before touching
+// global memory.
+inline bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("SVDQ_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
 }
 
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device) and

@@ -527,6 +527,11 @@ __global__ void __launch_bounds__(QCfg<ROT>::kThreads, 1)
     const float r = tid ? __frcp_rn(s) : 0.0f;
     tabs->srec[tid] = NEG ? make_float2(s, -r) : make_float2(-s, r);   // {-B, RN(1/B)}, B = -+s
   }
+  // Everything above overlaps the previous kernel's tail (programmatic
+  // dependent launch); nothing below runs before it has completed (its
+  // output may be this kernel's x, and it may still read the buffers this
+  // kernel writes).
+  griddep_wait();
   if (warp == kProducerWarp) {
     tmem_alloc(smem_u32(tmem_slot), tmem_cols);
     tmem_relinquish();
@@ -540,6 +545,7 @@ __global__ void __launch_bounds__(QCfg<ROT>::kThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  if (tid == 0) griddep_launch_dependents();
 
   int issued = 0;   // producer: loads issued
   if (warp == kProducerWarp) {
@@ -754,13 +760,15 @@ cudaError_t launch_impl(const CUtensorMap& tm_x, const CUtensorMap& tm_pdT, cons
   cfg.blockDim = dim3(QCfg<ROT>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = (unsigned)ksplit;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, tm_x, tm_pdT, tm_codes, p);
 }
 
