@@ -19,6 +19,7 @@ data path ("replicas only"); time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -60,6 +61,28 @@ def quant_bytes(M, K, R):
 def gemm_bytes(M, K, N, R):
     # codes + scales + L read, weights (codes + scales + proj_up + alpha) read, y written.
     return M * K / 2 + M * K / 16 + 2.0 * M * R + N * K / 2 + N * K / 16 + 2.0 * N * R + 4.0 * N + 2.0 * M * N
+
+
+def measured_traffic(workload, kernel):
+    """DRAM bytes (read + write) per launch from the ncu capture recorded in
+    profiles/traffic.json, or None when there is none or the kernel's source
+    has changed since it was taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)[workload][kernel]
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+                return None
+        return rec["dram_bytes_per_launch"]
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+def gemm_variant(ck):
+    """Which GEMM kernel the library picks for this layer (the same rule it applies at create time)."""
+    if os.environ.get("SVDQ_GEMM_TILE_N") == "128" or ck.R > 32:
+        return "gemm_nvfp4_lr_kernel, 128x128 tiles"
+    return "gemm_nvfp4_n256_kernel, 128x256 tiles, alpha folded into proj_up"
 
 
 class ClockSampler:
@@ -334,25 +357,18 @@ def run_ours(args, world, rank, local):
     kernels = {
         "quantize_act": {"us": us_q, "bound": "hbm", "algorithmic_bytes": quant_bytes(M, K, R),
                          "achieved_gbs": q_gbs, "frac_of_hbm": q_gbs / pk["hbm_gbs"]},
-        "gemm_nvfp4_lr": {"us": us_g, "bound": "tensor", "algorithmic_flops": g_flops, "achieved_tflops": g_tf,
-                          "frac_of_fp4": g_tf / fp4_peak, "algorithmic_bytes": gemm_bytes(M, K, N, R),
-                          "achieved_gbs": gemm_bytes(M, K, N, R) / (us_g * 1e-6) / 1e9},
+        "gemm_nvfp4": {"us": us_g, "bound": "tensor", "variant": gemm_variant(ck), "algorithmic_flops": g_flops,
+                       "achieved_tflops": g_tf, "frac_of_fp4": g_tf / fp4_peak,
+                       "algorithmic_bytes": gemm_bytes(M, K, N, R),
+                       "achieved_gbs": gemm_bytes(M, K, N, R) / (us_g * 1e-6) / 1e9},
     }
-    traffic = None
-    tf = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tf):
-        try:
-            with open(tf) as f:
-                traffic = json.load(f).get(ck.name, {}).get("gemm_nvfp4_lr")
-        except Exception:
-            traffic = None
     if us_g >= us_q:
-        roof = {"kernel": "gemm_nvfp4_lr", "bound": "tensor", "achieved": g_tf, "peak": fp4_peak,
-                "unit": "TFLOP/s", "frac": g_tf / fp4_peak, "traffic": traffic,
+        roof = {"kernel": "gemm_nvfp4 (" + gemm_variant(ck) + ")", "bound": "tensor", "achieved": g_tf, "peak": fp4_peak,
+                "unit": "TFLOP/s", "frac": g_tf / fp4_peak, "traffic": measured_traffic(ck.name, "gemm_nvfp4"),
                 "peak_source": f"{pk['source']} bf16 burst x {FP4_PER_BF16:g} (nominal FP4/BF16 ratio)"}
     else:
         roof = {"kernel": "quantize_act", "bound": "hbm", "achieved": q_gbs, "peak": pk["hbm_gbs"],
-                "unit": "GB/s", "frac": q_gbs / pk["hbm_gbs"], "traffic": None,
+                "unit": "GB/s", "frac": q_gbs / pk["hbm_gbs"], "traffic": measured_traffic(ck.name, "quantize_act"),
                 "peak_source": f"{pk['source']} copy bandwidth"}
     step_us = t_full_max / args.steps * 1e6
     line = {
