@@ -71,7 +71,8 @@ struct GParams {
   int M, N, R, k_tiles, ka_pad;   // k_tiles: K steps of 256 elements
   int m_tiles, n_tiles;   // n_tiles of 256 columns
   int lr_row_bytes;       // bytes per row of the L / proj_up' tiles in shared memory (32 or 64)
-  int y_vec;              // N % 8 == 0: y rows are 16-byte aligned, stored through the staging box
+  int y_mode;             // 2: 32-byte stores straight from registers (N % 16 == 0, y 32-byte aligned);
+                          // 1: through the staging box (N % 8 == 0); 0: element stores
 };
 
 // Shared-memory descriptor for a K-major tile with 32/64/128-byte rows (the
@@ -335,7 +336,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             o[2 * c + 1] =
                 pack_bf16x2(a4.z * __uint_as_float(acc[u][4 * c + 2]), a4.w * __uint_as_float(acc[u][4 * c + 3]));
           }
-          if (p.y_vec) {
+          if (p.y_mode == 2) {
+            // Each lane writes its row's 32 columns as two full 32-byte
+            // sectors; with N % 16 == 0 each 16-column store lies wholly inside
+            // or wholly outside the row.
+            if (m < p.M) {
+              __nv_bfloat16* dst = p.y + (size_t)m * p.N + nw + nl;
+              if (nw + nl + 16 <= p.N) st_global_v8(dst, o);
+              if (nw + nl + 32 <= p.N) st_global_v8(dst + 16, o + 8);
+            }
+          } else if (p.y_mode == 1) {
             // Row `lane` of a 64-column x 32-row box, 16-byte chunk c at
             // lane * 128 + ((c ^ (lane & 7)) * 16): conflict-free both when each
             // lane writes its row and when 8 lanes read one row back.
@@ -354,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (p.y_vec) {
+        if (p.y_mode == 1) {
           // Read the box back row-major (8 lanes x 16 bytes = one 128-byte row
           // segment) and store it coalesced.
           __syncwarp();
@@ -427,7 +437,13 @@ cudaError_t launch_gemm_nvfp4_n256(const GemmLaunch& L, cudaStream_t stream) {
   p.m_tiles = (L.M + BM - 1) / BM;
   p.n_tiles = (L.N + BN - 1) / BN;
   p.lr_row_bytes = row_bytes;
-  p.y_vec = (L.N % 8) == 0;
+  static const int y_env = [] {
+    const char* e = getenv("SVDQ_Y_STORE");
+    return e ? atoi(e) : -1;
+  }();
+  const bool v8_ok = (L.N % 16) == 0 && (reinterpret_cast<uintptr_t>(L.y) & 31u) == 0;
+  p.y_mode = v8_ok ? 2 : ((L.N % 8) == 0 ? 1 : 0);
+  if (y_env == 1 && (L.N % 8) == 0) p.y_mode = 1;   // tuning override: SVDQ_Y_STORE=1 forces the staging box
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = tiles < num_sms ? tiles : num_sms;
   cudaLaunchConfig_t cfg = {};
