@@ -438,6 +438,54 @@ __device__ __forceinline__ void smooth_cols(uint8_t* xs, const float4* lam4, con
   for (int rr = 0; rr < RPT; ++rr) write_back_bf16(xs, r0 + kColRowStride * rr, 2 * j, v[rr]);
 }
 
+// smooth_cols for the last, ragged row tile: the thread's rows are handled one
+// at a time and rows at or beyond `nvalid` (they do not exist; their shared
+// memory was zero-filled by the TMA load) are skipped, with zero codes and
+// scales staged for them.
+template <bool NEG>
+__device__ __noinline__ void smooth_cols_partial(uint8_t* xs, const float4* lam4, const float2* srec, float y6, int t,
+                                                 int nvalid, uint32_t (&cw)[kColRowsPerThread][2],
+                                                 uint32_t (&sb)[kColRowsPerThread]) {
+  const int j = t & 7, r0 = t >> 3;
+  uint64_t nb[8], yb[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 l = lam4[8 * i + j];
+    nb[i] = pk2(l.x, l.y);
+    yb[i] = pk2(l.z, l.w);
+  }
+#pragma unroll
+  for (int rr = 0; rr < kColRowsPerThread; ++rr) {
+    const int row = r0 + kColRowStride * rr;
+    cw[rr][0] = cw[rr][1] = 0u;
+    sb[rr] = 0u;
+    if (row >= nvalid) continue;
+    const uint4 p0 = *reinterpret_cast<const uint4*>(xs + xoff(row, 2 * j));
+    const uint4 p1 = *reinterpret_cast<const uint4*>(xs + xoff(row, 2 * j + 1));
+    const uint32_t xin[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    uint64_t v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      v[i] = NEG ? div_mk2(bf16x2_to_f2(xin[i]), nb[i], yb[i]) : div_rn2(bf16x2_to_f2(xin[i]), nb[i], yb[i]);
+    const float amax = amax8(v);
+    if (amax < 3.0e38f) {
+      sb[rr] = quant_block<NEG>(v, amax, srec, y6, cw[rr][0], cw[rr][1]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float s0 = NEG ? lo2(nb[i]) : -lo2(nb[i]), s1 = NEG ? hi2(nb[i]) : -hi2(nb[i]);
+        v[i] = pk2(__fdiv_rn(__uint_as_float(xin[i] << 16), s0), __fdiv_rn(__uint_as_float(xin[i] & 0xFFFF0000u), s1));
+      }
+      sb[rr] = quant_block_slow(v, cw[rr][0], cw[rr][1]);
+      if (NEG) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] ^= 0x8000000080000000ull;
+      }
+    }
+    write_back_bf16(xs, row, 2 * j, v);
+  }
+}
+
 __device__ __forceinline__ void stage_cols(uint8_t* cst, uint8_t* sst, int t,
                                            const uint32_t (&cw)[kColRowsPerThread][2],
                                            const uint32_t (&sb)[kColRowsPerThread]) {
@@ -610,18 +658,34 @@ __global__ void __launch_bounds__(QCfg<ROT>::kThreads, 1)
     // compute warps: the chunk's 128 rows x 128 channels
     const float y6 = __frcp_rn(6.0f);
     const int row2 = tid >> 1, q = tid & 1;      // rotated mapping: two threads per row
+    const int nvalid = p.M - m0;                 // rows of this tile that exist (>= 1)
     for (int i = 0; i < nch; ++i) {
       const int s = i % p.stages;
-      if (!wait_bounded(smem_u32(&full[s]), (i / p.stages) & 1, abort_flag, p.err, kErrQuantTimeout)) break;
+      // Warp-uniform outcome: the rotated path uses full-warp shuffles.
+      if (!__all_sync(0xffffffffu, wait_bounded(smem_u32(&full[s]), (i / p.stages) & 1, abort_flag, p.err,
+                                                kErrQuantTimeout)))
+        break;
       const int kc = (c_begin + i) * kChunk;
       uint8_t* xs = X + s * kXStageBytes;
       const float4* lam = reinterpret_cast<const float4*>(LAM + s * kLamStageBytes);
       uint32_t cw8[8], sbytes = 0;                 // rotated mapping
       uint32_t cw[kColRowsPerThread][2], sb[kColRowsPerThread];   // column mapping
-      if (ROT)
-        rotate_half(xs, lam, tabs->srec, y6, row2, q, cw8, sbytes);
-      else
+      if (ROT) {
+        // rotate_half exchanges values between lane pairs with full-warp
+        // shuffles, so only a whole warp may skip: all 16 of its rows lie
+        // beyond M (rows beyond M that a warp does process are zero-filled
+        // and rotate to zero).
+        if ((row2 & ~15) < nvalid) {
+          rotate_half(xs, lam, tabs->srec, y6, row2, q, cw8, sbytes);
+        } else {                     // no row of this warp exists: zeros staged
+#pragma unroll
+          for (int c = 0; c < 8; ++c) cw8[c] = 0u;
+        }
+      } else if (nvalid >= kRows) {
         smooth_cols<NEG>(xs, lam, tabs->srec, y6, tid, cw, sb);
+      } else {
+        smooth_cols_partial<NEG>(xs, lam, tabs->srec, y6, tid, nvalid, cw, sb);
+      }
       if (TILED) {
         // The stores that last read this stage's staging buffers finished
         // before the stage was released for this chunk's load.
@@ -664,7 +728,8 @@ __global__ void __launch_bounds__(QCfg<ROT>::kThreads, 1)
   const int rows_per = kRows / p.ksplit;
   if (want_lr && tid < kRows) {
     // warps 0-3 read TMEM lane quadrants 0-3: thread tid owns row tid.
-    const bool ok = wait_bounded(smem_u32(done), 0, abort_flag, p.err, kErrQuantTimeout);
+    // Warp-uniform outcome: the TMEM loads below are warp-wide instructions.
+    const bool ok = __all_sync(0xffffffffu, wait_bounded(smem_u32(done), 0, abort_flag, p.err, kErrQuantTimeout));
     tc_fence_after_sync();
     const int row = tid, m = m0 + row;
     const uint32_t owner = (uint32_t)(row / rows_per);

@@ -28,6 +28,7 @@ struct svdq_linear {
   __nv_bfloat16* pu_fold; // proj_up' = bf16(proj_up / alpha) (N, R); proj_up where alpha = 0
   float* alpha_fold;      // (roundup(N, 256)) alpha, or 1 where alpha = 0
   bool n256;              // GEMM on 128 x 256 tiles with alpha folded into proj_up
+  bool splitk;            // few rows: split-K GEMM over a cluster (unless SVDQ_SPLITK=0 at create)
   int lr_row_bytes;       // 128 x 256 GEMM: bytes per row of its L / proj_up' tiles
   unsigned* err;          // device error word
   CUtensorMap tm_b, tm_pdT, tm_pu;
@@ -350,6 +351,8 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
     const char* env = std::getenv("SVDQ_GEMM_TILE_N");
     const bool force128 = env && std::strcmp(env, "128") == 0;
     h->n256 = !(bad & 8u) && d->R <= 32 && !force128;
+    const char* sk = std::getenv("SVDQ_SPLITK");
+    h->splitk = !(sk && sk[0] == '0');
     h->lr_row_bytes = svdq::gemm_n256_lr_row_bytes(d->R);
   }
 #undef CREATE_CUDA
@@ -363,10 +366,11 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
   if ((s = make_tmap(&h->tm_pu, h->pu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d->R, d->N, (uint64_t)d->R * 2, 64, 128)) !=
       SVDQ_OK)
     return fail(s);
+  // 256-row weight boxes: the 128 x 256 kernel and the split-K kernel for few rows.
+  if ((s = make_tmap(&h->tm_b256, h->qw, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->Kp / 2, d->N, h->Kp / 2, 128, 256)) !=
+      SVDQ_OK)
+    return fail(s);
   if (h->n256) {
-    if ((s = make_tmap(&h->tm_b256, h->qw, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->Kp / 2, d->N, h->Kp / 2, 128, 256)) !=
-        SVDQ_OK)
-      return fail(s);
     if ((s = make_tmap(&h->tm_pu_fold, h->pu_fold, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d->R, d->N, (uint64_t)d->R * 2,
                        h->lr_row_bytes / 2, 256, lr_swizzle(h->lr_row_bytes))) != SVDQ_OK)
       return fail(s);
@@ -463,6 +467,17 @@ svdq_status forward_quantize(const svdq_linear* h, const void* x, int M, void* w
   return SVDQ_OK;
 }
 
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
 svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, cudaStream_t stream) {
   const WsLayout w = ws_layout(h, M);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -480,6 +495,15 @@ svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, 
   g.R = h->R;
   g.k_tiles = h->k_tiles;
   g.ka_pad = h->ka_pad;
+  // Few rows: split K over a cluster so the weight read is spread over the GPU.
+  const int S = h->splitk ? svdq::gemm_splitk_slices(M, h->N, h->R, h->k_tiles, num_sms()) : 1;
+  if (S > 1) {
+    g.tm_b = h->tm_b256;
+    g.alpha = h->alpha;
+    cudaError_t e = svdq::launch_gemm_nvfp4_splitk(g, ws + w.lr, h->pu, S, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+    return SVDQ_OK;
+  }
   if (h->n256) {
     g.tm_b = h->tm_b256;
     if ((s = make_tmap(&g.tm_l, ws + w.lr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->R, M, (uint64_t)h->R * 2,

@@ -58,6 +58,15 @@ cudaError_t launch_gemm_nvfp4_lr(const GemmLaunch& p, cudaStream_t stream);
 //   alpha  alpha' (alpha, or 1 where alpha is 0)
 // Requires R <= 32 (the L / proj_up' tile must fit beside the ring and staging).
 int gemm_n256_lr_row_bytes(int R);
+
+// Split-K variant for few rows (tiles too few to fill the GPU): 128 x 256
+// tiles, each tile's K range split over an S-CTA cluster (S = 2, 4, 8);
+// GemmLaunch as for the 128 x 256 kernel (tm_b box {128, 256}) but with the
+// plain alpha; the rank-R term is read from `lowrank` (M, R) and `proj_up`
+// (N, R) directly.  gemm_splitk_slices returns the S to use (1: do not split).
+int gemm_splitk_slices(int M, int N, int R, int k_tiles, int num_sms);
+cudaError_t launch_gemm_nvfp4_splitk(const GemmLaunch& p, const void* lowrank, const void* proj_up, int S,
+                                     cudaStream_t stream);
 cudaError_t launch_gemm_nvfp4_n256(const GemmLaunch& p, cudaStream_t stream);
 
 }  // namespace svdq

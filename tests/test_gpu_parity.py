@@ -252,6 +252,16 @@ def test_full_workload_parity(name):
 
 # ------------------------------------------------------------------ ragged shapes and edge cases
 
+def _select_gemm(kernel, monkeypatch):
+    """"auto": the library's choice (split-K over a cluster for few rows, else
+    128 x 256 tiles with alpha folded when R <= 32, else 128 x 128);
+    "n256" / "n128": the persistent kernels without split-K."""
+    if kernel in ("n256", "n128"):
+        monkeypatch.setenv("SVDQ_SPLITK", "0")
+    if kernel == "n128":
+        monkeypatch.setenv("SVDQ_GEMM_TILE_N", "128")
+
+
 @pytest.mark.parametrize("M,K,N,R,rot", [
     (1, 256, 256, 32, 0),
     (3, 48, 8, 16, 0),          # K < one chunk, N < one tile
@@ -261,13 +271,12 @@ def test_full_workload_parity(name):
     (130, 384, 256, 32, 128),   # rotation, K = 3 rotation blocks
     (64, 2048, 640, 64, 128),
     (300, 4096, 128, 32, 0),    # split-K cluster reduction with ragged rows
+    (40, 1008, 300, 128, 0),    # few rows: split-K GEMM, ragged N, R = 128
 ])
-@pytest.mark.parametrize("tile", ["auto", "128"])
-def test_ragged_shapes(M, K, N, R, rot, tile, monkeypatch):
-    """Both GEMM kernels: "auto" takes the 128 x 256 tiles with alpha folded
-    into proj_up where R <= 64, "128" forces the 128 x 128 kernel."""
-    if tile == "128":
-        monkeypatch.setenv("SVDQ_GEMM_TILE_N", "128")
+@pytest.mark.parametrize("kernel", ["auto", "n256", "n128"])
+def test_ragged_shapes(M, K, N, R, rot, kernel, monkeypatch):
+    """Every GEMM kernel on every ragged shape (see _select_gemm)."""
+    _select_gemm(kernel, monkeypatch)
     ck = synthetic.make_checkpoint(M, K, N, R, seed=M + K + N + R, rotate_block=rot, dense_weight=bool(rot),
                                    wcscales="uniform", wtscale=0.75, name=f"ragged_{M}x{K}x{N}_r{R}_rot{rot}")
     layer = make_layer(ck)
@@ -276,12 +285,11 @@ def test_ragged_shapes(M, K, N, R, rot, tile, monkeypatch):
     check_forward(layer, ck)
 
 
-@pytest.mark.parametrize("tile", ["auto", "128"])
-def test_zero_alpha_columns(tile, monkeypatch):
-    """Columns with wcscales = 0 reduce to the rank-R branch alone, in both
-    GEMM kernels (the folded one gives them alpha' = 1 and zero weight scales)."""
-    if tile == "128":
-        monkeypatch.setenv("SVDQ_GEMM_TILE_N", "128")
+@pytest.mark.parametrize("kernel", ["auto", "n256", "n128"])
+def test_zero_alpha_columns(kernel, monkeypatch):
+    """Columns with wcscales = 0 reduce to the rank-R branch alone, in every
+    GEMM kernel (the folded one gives them alpha' = 1 and zero weight scales)."""
+    _select_gemm(kernel, monkeypatch)
     ck = synthetic.make_checkpoint(150, 512, 520, 32, seed=12, wcscales="uniform",
                                    name="zero_alpha_150x512x520_r32")
     zero_cols = np.array([0, 1, 127, 128, 255, 256, 300, 511, 512, 519])
@@ -294,9 +302,12 @@ def test_zero_alpha_columns(tile, monkeypatch):
     assert_y_close(y[:, zero_cols], lr[:, zero_cols], "zero-alpha columns")
 
 
-def test_unfoldable_alpha_takes_plain_epilogue():
+def test_unfoldable_alpha_takes_plain_epilogue(monkeypatch):
     """wtscale = 2^-30 is outside the range where proj_up / alpha keeps bf16
-    precision, so the layer keeps alpha in the epilogue; results still match."""
+    precision, so the layer keeps alpha in the epilogue (the 128 x 128 kernel:
+    split-K, which also applies alpha in its epilogue, is switched off here);
+    results still match."""
+    monkeypatch.setenv("SVDQ_SPLITK", "0")
     ck = synthetic.make_checkpoint(140, 512, 384, 32, seed=13, wcscales="uniform", wtscale=2.0 ** -30,
                                    name="tiny_alpha_140x512x384_r32")
     layer = make_layer(ck)
