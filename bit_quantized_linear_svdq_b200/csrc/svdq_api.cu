@@ -31,6 +31,9 @@ struct svdq_linear {
   bool splitk;            // few rows: split-K GEMM over a cluster (unless SVDQ_SPLITK=0 at create)
   int lr_row_bytes;       // 128 x 256 GEMM: bytes per row of its L / proj_up' tiles
   unsigned* err;          // device error word
+  // svdq_linear_forward_host: copy streams and events of its row-chunk pipeline.
+  cudaStream_t s_in, s_out;
+  cudaEvent_t ev_start, ev_out, ev_in[16], ev_comp[16];
   CUtensorMap tm_b, tm_pdT, tm_pu;
   CUtensorMap tm_b256, tm_pu_fold;
 };
@@ -216,6 +219,14 @@ void free_handle(svdq_linear* h) {
   cudaFree(h->pu_fold);
   cudaFree(h->alpha_fold);
   cudaFree(h->err);
+  if (h->s_in) cudaStreamDestroy(h->s_in);
+  if (h->s_out) cudaStreamDestroy(h->s_out);
+  if (h->ev_start) cudaEventDestroy(h->ev_start);
+  if (h->ev_out) cudaEventDestroy(h->ev_out);
+  for (int i = 0; i < 16; ++i) {
+    if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+    if (h->ev_comp[i]) cudaEventDestroy(h->ev_comp[i]);
+  }
   delete h;
 }
 
@@ -314,6 +325,14 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
   CREATE_CUDA(cudaMalloc(&h->pu_fold, (size_t)d->N * d->R * 2));
   CREATE_CUDA(cudaMalloc(&h->alpha_fold, (size_t)Npad256 * sizeof(float)));
   CREATE_CUDA(cudaMalloc(&h->err, 2 * sizeof(unsigned)));   // [0] device error word, [1] create-time checks
+  CREATE_CUDA(cudaStreamCreateWithFlags(&h->s_in, cudaStreamNonBlocking));
+  CREATE_CUDA(cudaStreamCreateWithFlags(&h->s_out, cudaStreamNonBlocking));
+  CREATE_CUDA(cudaEventCreateWithFlags(&h->ev_start, cudaEventDisableTiming));
+  CREATE_CUDA(cudaEventCreateWithFlags(&h->ev_out, cudaEventDisableTiming));
+  for (int i = 0; i < 16; ++i) {
+    CREATE_CUDA(cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming));
+    CREATE_CUDA(cudaEventCreateWithFlags(&h->ev_comp[i], cudaEventDisableTiming));
+  }
   CREATE_CUDA(cudaMemsetAsync(h->err, 0, 2 * sizeof(unsigned), stream));
 
   CREATE_CUDA(cudaMemset2DAsync(h->qw, h->Kp / 2, 0, h->Kp / 2, d->N, stream));
@@ -559,12 +578,59 @@ svdq_status svdq_linear_forward_host(const svdq_linear* h, const void* x_host, i
   if (M == 0) return SVDQ_OK;
   if (!x_host || !y_host) return SVDQ_ERR_INVALID_ARG;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-  SVDQ_CUDA(cudaMemcpyAsync(x_dev, x_host, (size_t)M * h->K * 2, cudaMemcpyHostToDevice, stream));
-  svdq_status s = svdq_linear_forward(h, x_dev, M, y_dev, workspace, stream_);
-  if (s != SVDQ_OK) return s;
-  SVDQ_CUDA(cudaMemcpyAsync(y_host, y_dev, (size_t)M * h->N * 2, cudaMemcpyDeviceToHost, stream));
+  // Row chunks: one for M < 1024, else six with boundaries at 1/16, 4/16,
+  // 8/16, 12/16 and 15/16 of M (rounded down to 128 rows).  The host-to-device
+  // copy of chunk i+1 (stream s_in), the layer on chunk i (the caller's
+  // stream) and the device-to-host copy of chunk i-1 (stream s_out) run at the
+  // same time; the short first and last chunks keep the start (copy in, no
+  // copy out yet) and the end (copy out only) short.  Few large copies: PCIe
+  // moves less in both directions together when the copies are many and
+  // small.  Chunks run in order on the caller's stream and share the
+  // workspace.  Every chunk but the last is a multiple of 128 rows and the
+  // last has at least M/16 rows, so no chunk takes the few-row GEMM when M
+  // does not.
+  int bounds[7];
+  int n_chunks = 0;
+  bounds[0] = 0;
+  if (M < 1024) {
+    bounds[++n_chunks] = M;
+  } else {
+    static const int cum16[5] = {1, 4, 8, 12, 15};
+    for (int i = 0; i < 5; ++i) {
+      const int b = (int)(((int64_t)M * cum16[i] / 16) & ~127);
+      if (b > bounds[n_chunks]) bounds[++n_chunks] = b;
+    }
+    bounds[++n_chunks] = M;
+  }
+  const size_t xrow = (size_t)h->K * 2, yrow = (size_t)h->N * 2;
+  SVDQ_CUDA(cudaEventRecord(h->ev_start, stream));          // work queued before this call
+  SVDQ_CUDA(cudaStreamWaitEvent(h->s_in, h->ev_start, 0));
+  SVDQ_CUDA(cudaStreamWaitEvent(h->s_out, h->ev_start, 0));
+  for (int c = 0; c < n_chunks; ++c) {
+    const int r0 = bounds[c], rc = bounds[c + 1] - bounds[c];
+    SVDQ_CUDA(cudaMemcpyAsync(static_cast<uint8_t*>(x_dev) + r0 * xrow, static_cast<const uint8_t*>(x_host) + r0 * xrow,
+                              (size_t)rc * xrow, cudaMemcpyHostToDevice, h->s_in));
+    SVDQ_CUDA(cudaEventRecord(h->ev_in[c], h->s_in));
+  }
+  svdq_status s = SVDQ_OK;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int r0 = bounds[c], rc = bounds[c + 1] - bounds[c];
+    SVDQ_CUDA(cudaStreamWaitEvent(stream, h->ev_in[c], 0));
+    s = svdq_linear_forward(h, static_cast<const uint8_t*>(x_dev) + r0 * xrow, rc,
+                            static_cast<uint8_t*>(y_dev) + r0 * yrow, workspace, stream_);
+    if (s != SVDQ_OK) break;
+    SVDQ_CUDA(cudaEventRecord(h->ev_comp[c], stream));
+    SVDQ_CUDA(cudaStreamWaitEvent(h->s_out, h->ev_comp[c], 0));
+    SVDQ_CUDA(cudaMemcpyAsync(static_cast<uint8_t*>(y_host) + r0 * yrow, static_cast<const uint8_t*>(y_dev) + r0 * yrow,
+                              (size_t)rc * yrow, cudaMemcpyDeviceToHost, h->s_out));
+  }
+  // The caller's stream ends after every copy (also on an error above).
+  SVDQ_CUDA(cudaEventRecord(h->ev_out, h->s_out));
+  SVDQ_CUDA(cudaStreamWaitEvent(stream, h->ev_out, 0));
+  SVDQ_CUDA(cudaEventRecord(h->ev_start, h->s_in));
+  SVDQ_CUDA(cudaStreamWaitEvent(stream, h->ev_start, 0));
   SVDQ_CUDA(cudaStreamSynchronize(stream));
-  return SVDQ_OK;
+  return s;
 }
 
 svdq_status svdq_device_status(const svdq_linear* h, int* flags) {

@@ -144,9 +144,11 @@ SVDQ_API svdq_status svdq_linear_forward_gemm(const svdq_linear* h, int M, void*
 /*
  * svdq_linear_forward_host -- end-to-end call on HOST buffers: copies x_host
  * (M, K bf16) to x_dev, runs svdq_linear_forward into y_dev, copies y_dev to
- * y_host (M, N bf16) and synchronizes `stream` before returning.  Host
- * buffers should be pinned for full copy bandwidth.  x_dev / y_dev /
- * workspace are caller-owned device buffers as in svdq_linear_forward.
+ * y_host (M, N bf16) and synchronizes `stream` before returning.  The copies
+ * and the layer are pipelined over row chunks (two copy streams owned by the
+ * handle), so calls on one handle must not overlap.  Host buffers should be
+ * pinned (required for the overlap).  x_dev / y_dev / workspace are
+ * caller-owned device buffers as in svdq_linear_forward.
  */
 SVDQ_API svdq_status svdq_linear_forward_host(const svdq_linear* h, const void* x_host, int M, void* y_host,
                                      void* x_dev, void* y_dev, void* workspace, void* stream);

@@ -271,7 +271,7 @@ def _select_gemm(kernel, monkeypatch):
     (130, 384, 256, 32, 128),   # rotation, K = 3 rotation blocks
     (64, 2048, 640, 64, 128),
     (300, 4096, 128, 32, 0),    # split-K cluster reduction with ragged rows
-    (40, 1008, 300, 128, 0),    # few rows: split-K GEMM, ragged N, R = 128
+    (24, 1008, 300, 128, 0),    # few rows: split-K GEMM, ragged N, R = 128
 ])
 @pytest.mark.parametrize("kernel", ["auto", "n256", "n128"])
 def test_ragged_shapes(M, K, N, R, rot, kernel, monkeypatch):
@@ -348,19 +348,30 @@ def test_zero_rows_is_noop():
     assert S.svdq_workspace_bytes(layer.handle, 0) == 0
 
 
-def test_forward_host_matches_device_path():
-    ck = synthetic.make_checkpoint(64, 512, 384, 32, seed=9)
+@pytest.mark.parametrize("M", [64, 300, 1000, 1030, 4100])
+def test_forward_host_matches_device_path(M):
+    """The host-buffer call pipelines its copies over row chunks: one chunk
+    (the device call itself, so bit for bit the same y) for M < 1024, six from
+    M = 1024 on.  A chunk's quantizer may split K over more CTAs than the whole
+    call's, which changes the fp32 summation order of L = x_hat proj_down, so
+    chunked results are held to the oracle's y tolerance instead."""
+    ck = synthetic.make_checkpoint(M, 512, 384, 32, seed=9)
     layer = make_layer(ck)
     x = dev_bf16(ck.x)
     y_dev_ref = layer.forward(x).clone()
     xh = x.cpu().pin_memory()
-    yh = torch.empty((64, 384), dtype=torch.bfloat16).pin_memory()
+    yh = torch.full((M, 384), float("nan"), dtype=torch.bfloat16).pin_memory()
     xd = torch.empty_like(x)
-    yd = torch.empty((64, 384), dtype=torch.bfloat16, device="cuda")
-    ws = layer.workspace(64)
-    S.svdq_linear_forward_host(layer.handle, xh.data_ptr(), 64, yh.data_ptr(), xd.data_ptr(), yd.data_ptr(),
+    yd = torch.empty((M, 384), dtype=torch.bfloat16, device="cuda")
+    ws = layer.workspace(M)
+    S.svdq_linear_forward_host(layer.handle, xh.data_ptr(), M, yh.data_ptr(), xd.data_ptr(), yd.data_ptr(),
                                ws.data_ptr())
-    assert torch.equal(yh, y_dev_ref.cpu())
+    assert layer.device_status() == 0
+    if M < 1024:
+        assert torch.equal(yh, y_dev_ref.cpu())
+    else:
+        assert not torch.isnan(yh.float()).any()
+        assert_y_close(host_bf16_to_f64(yh), O.linear_forward(ck), ck.name)
 
 
 def test_runtime_argument_errors():
