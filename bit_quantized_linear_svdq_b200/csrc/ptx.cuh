@@ -313,6 +313,77 @@ __host__ __device__ constexpr uint32_t idesc_nvfp4(uint32_t m, uint32_t n) {
 }
 
 // --------------------------------------------------------------------------
+// CTA pairs (tcgen05 .cta_group::2): one MMA spans the tensor cores of two
+// SMs of a 2-CTA cluster.  Every tcgen05 instruction of a kernel that uses
+// pairs takes .cta_group::2.
+// --------------------------------------------------------------------------
+// Both CTAs of the pair, from the same warp, with the same dst offset.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Arrive once, when every pair MMA this thread issued has completed, on the
+// mbarrier at shared offset `bar` in each CTA of `cta_mask`.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          bar),
+      "h"(cta_mask)
+      : "memory");
+}
+// Pair MMA, bf16 inputs (M = 256: A rows 0-127 from this CTA's shared memory,
+// 128-255 from the peer's at the same offset; B's N rows split the same way).
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Pair MMA, packed E2M1 with one UE4M3 scale per 16 K elements; each CTA's
+// TMEM holds the A scales of its own rows and the B scales of all N columns.
+__device__ __forceinline__ void mma_nvfp4_pair(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+// 2-D tiled load into this CTA's shared memory whose bytes complete on the
+// mbarrier at the same offset in the pair's even CTA (bit 24 of a shared
+// address selects the CTA within the pair).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* m, uint32_t bar, int32_t c0,
+                                                 int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar & 0xFEFFFFFFu), "r"(c0), "r"(c1)
+      : "memory");
+}
+// Arrive on the mbarrier at shared offset `bar` of cluster CTA `rank`.  Only
+// tensor-memory work is ordered through these arrivals (by the tcgen05
+// fences around them), so the default semantics suffice.
+__device__ __forceinline__ void mbar_arrive_on(uint32_t bar, uint32_t rank) {
+  asm volatile(
+      "{\n\t.reg .b32 ra;\n\t"
+      "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+      "mbarrier.arrive.shared::cluster.b64 _, [ra];\n\t}" ::"r"(bar),
+      "r"(rank)
+      : "memory");
+}
+
+// --------------------------------------------------------------------------
 // clusters
 // --------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {

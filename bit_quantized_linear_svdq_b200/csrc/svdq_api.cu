@@ -29,13 +29,14 @@ struct svdq_linear {
   float* alpha_fold;      // (roundup(N, 256)) alpha, or 1 where alpha = 0
   bool n256;              // GEMM on 128 x 256 tiles with alpha folded into proj_up
   bool splitk;            // few rows: split-K GEMM over a cluster (unless SVDQ_SPLITK=0 at create)
+  bool pair;              // more than 128 rows: 256 x 256 tiles on CTA pairs (unless SVDQ_GEMM_PAIR=0 at create)
   int lr_row_bytes;       // 128 x 256 GEMM: bytes per row of its L / proj_up' tiles
   unsigned* err;          // device error word
   // svdq_linear_forward_host: copy streams and events of its row-chunk pipeline.
   cudaStream_t s_in, s_out;
   cudaEvent_t ev_start, ev_out, ev_in[16], ev_comp[16];
   CUtensorMap tm_b, tm_pdT, tm_pu;
-  CUtensorMap tm_b256, tm_pu_fold;
+  CUtensorMap tm_b256, tm_pu_fold, tm_pu_fold128;
 };
 
 namespace {
@@ -372,6 +373,9 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
     h->n256 = !(bad & 8u) && d->R <= 32 && !force128;
     const char* sk = std::getenv("SVDQ_SPLITK");
     h->splitk = !(sk && sk[0] == '0');
+    // 256 x 256 pair tiles (2-CTA clusters) unless SVDQ_GEMM_PAIR=0.
+    const char* pr = std::getenv("SVDQ_GEMM_PAIR");
+    h->pair = h->n256 && !(pr && pr[0] == '0');
     h->lr_row_bytes = svdq::gemm_n256_lr_row_bytes(d->R);
   }
 #undef CREATE_CUDA
@@ -392,6 +396,9 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
   if (h->n256) {
     if ((s = make_tmap(&h->tm_pu_fold, h->pu_fold, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d->R, d->N, (uint64_t)d->R * 2,
                        h->lr_row_bytes / 2, 256, lr_swizzle(h->lr_row_bytes))) != SVDQ_OK)
+      return fail(s);
+    if ((s = make_tmap(&h->tm_pu_fold128, h->pu_fold, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d->R, d->N,
+                       (uint64_t)d->R * 2, h->lr_row_bytes / 2, 128, lr_swizzle(h->lr_row_bytes))) != SVDQ_OK)
       return fail(s);
   }
   *out = h;
@@ -501,6 +508,7 @@ svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, 
   const WsLayout w = ws_layout(h, M);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   svdq::GemmLaunch g;
+  std::memset(&g, 0, sizeof(g));
   svdq_status s;
   if ((s = make_tmap(&g.tm_a, ws + w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->Kp / 2, M, h->Kp / 2, 128, 128)) !=
       SVDQ_OK)
@@ -520,6 +528,20 @@ svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, 
     g.tm_b = h->tm_b256;
     g.alpha = h->alpha;
     cudaError_t e = svdq::launch_gemm_nvfp4_splitk(g, ws + w.lr, h->pu, S, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+    return SVDQ_OK;
+  }
+  if (h->pair && M > 128 && svdq::gemm_pair_available(h->R)) {
+    g.tm_b = h->tm_b;
+    if ((s = make_tmap(&g.tm_l, ws + w.lr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->R, M, (uint64_t)h->R * 2,
+                       h->lr_row_bytes / 2, 128, lr_swizzle(h->lr_row_bytes))) != SVDQ_OK)
+      return s;
+    g.tm_pu = h->tm_pu_fold128;
+    g.alpha = h->alpha_fold;
+    if (h->N % 8 == 0 &&
+        (s = make_tmap(&g.tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->N, M, (uint64_t)h->N * 2, 64, 32)) != SVDQ_OK)
+      return s;
+    cudaError_t e = svdq::launch_gemm_nvfp4_pair(g, stream);
     if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
     return SVDQ_OK;
   }

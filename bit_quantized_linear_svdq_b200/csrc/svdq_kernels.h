@@ -38,6 +38,7 @@ struct GemmLaunch {
   CUtensorMap tm_b;         // weight codes u8 (N, Kp/2): box {128, 128}, 128B swizzle
   CUtensorMap tm_l;         // L bf16 (M, R): box {64, 128}, 128B swizzle
   CUtensorMap tm_pu;        // proj_up bf16 (N, R): box {64, 128}, 128B swizzle
+  CUtensorMap tm_y;         // pair kernel with N % 8 == 0: y bf16 (M, N), box {64, 32}, 128B swizzle
   const uint8_t* sfa;       // activation scale tiles
   const uint8_t* sfb;       // weight scale tiles
   const float* alpha;       // (N padded to 128) wcscales * wtscale
@@ -68,5 +69,15 @@ int gemm_splitk_slices(int M, int N, int R, int k_tiles, int num_sms);
 cudaError_t launch_gemm_nvfp4_splitk(const GemmLaunch& p, const void* lowrank, const void* proj_up, int S,
                                      cudaStream_t stream);
 cudaError_t launch_gemm_nvfp4_n256(const GemmLaunch& p, cudaStream_t stream);
+
+// The same product on 256 x 256 tiles, each computed by a 2-CTA cluster with
+// pair (cta_group::2) MMAs; alpha folded as for the 128 x 256 kernel.  The
+// GemmLaunch fields then hold:
+//   tm_b   weight codes: box {128, 128} (each CTA loads its half of the tile)
+//   tm_l   L: box {lr_row_bytes / 2, 128}, swizzle of lr_row_bytes
+//   tm_pu  proj_up' (N, R): box {lr_row_bytes / 2, 128}, same swizzle
+// gemm_pair_available: R <= 32 and at least one pair fits on the device.
+bool gemm_pair_available(int R);
+cudaError_t launch_gemm_nvfp4_pair(const GemmLaunch& p, cudaStream_t stream);
 
 }  // namespace svdq

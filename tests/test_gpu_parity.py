@@ -254,10 +254,12 @@ def test_full_workload_parity(name):
 
 def _select_gemm(kernel, monkeypatch):
     """"auto": the library's choice (split-K over a cluster for few rows, else
-    128 x 256 tiles with alpha folded when R <= 32, else 128 x 128);
-    "n256" / "n128": the persistent kernels without split-K."""
+    with alpha folded when R <= 32: 256 x 256 tiles on CTA pairs above 128
+    rows, 128 x 256 tiles otherwise; else 128 x 128); "n256" / "n128": the
+    one-CTA persistent kernels without split-K."""
     if kernel in ("n256", "n128"):
         monkeypatch.setenv("SVDQ_SPLITK", "0")
+        monkeypatch.setenv("SVDQ_GEMM_PAIR", "0")
     if kernel == "n128":
         monkeypatch.setenv("SVDQ_GEMM_TILE_N", "128")
 
@@ -272,6 +274,8 @@ def _select_gemm(kernel, monkeypatch):
     (64, 2048, 640, 64, 128),
     (300, 4096, 128, 32, 0),    # split-K cluster reduction with ragged rows
     (24, 1008, 300, 128, 0),    # few rows: split-K GEMM, ragged N, R = 128
+    (2048, 256, 2560, 32, 0),   # more 256 x 256 tiles than CTA pairs: two tiles per pair
+    (260, 512, 300, 32, 0),     # pair tiles with N % 8 != 0: element stores instead of TMA
 ])
 @pytest.mark.parametrize("kernel", ["auto", "n256", "n128"])
 def test_ragged_shapes(M, K, N, R, rot, kernel, monkeypatch):
