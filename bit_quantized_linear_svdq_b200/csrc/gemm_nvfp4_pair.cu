@@ -85,6 +85,18 @@ struct PParams {
   int y_mode;             // 3: through shared-memory boxes and TMA stores (N % 8 == 0); 0: element stores
 };
 
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+// Two fp32 products, each rounded once (as two fmul.rn).
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 __device__ __forceinline__ uint64_t sdesc_rows(uint32_t saddr, int row_bytes) {
   const uint64_t layout = row_bytes == 128 ? 2ull : (row_bytes == 64 ? 4ull : 6ull);
   return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(16u >> 4) << 16) |
@@ -302,8 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // Epilogue warp e: TMEM lane quadrant q = warp & 3 (rows 32q..32q+31 of
     // this CTA's half of the tile), all 256 columns, in 64-column chunks.
-    // With y_mode 3 a chunk goes, as bf16, into one of the warp's two
-    // 64-column x 32-row boxes (128-byte rows, 16-byte chunk c of row r at
+    // Chunk pc + 1 is read from TMEM while chunk pc is converted.  With
+    // y_mode 3 a chunk goes, as bf16, into one of the warp's two 64-column x
+    // 32-row boxes (128-byte rows, 16-byte chunk c of row r at
     // r * 128 + (c ^ (r % 8)) * 16: the TMA 128-byte swizzle, conflict-free for
     // the row-per-lane writes) and leaves with a TMA store.  Nothing waits for
     // global memory before the accumulator is released: the release follows
@@ -333,14 +346,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool w = wait_bounded(smem_u32(acc_full), it & 1, abort_flag, p.err, kErrGemmTimeout);
       if (!__all_sync(0xffffffffu, w)) break;
       tc_fence_after_sync();
-#pragma unroll 1
+      // Chunk pc + 1 is read from TMEM while chunk pc is converted.
+      uint32_t acc[2][2][32];
+      tmem_ld32(lane_base, acc[0][0]);
+      tmem_ld32(lane_base + 32, acc[0][1]);
+#pragma unroll
       for (int pc = 0; pc < kEpiCols / 64; ++pc) {
         const int nl0 = 64 * pc;
-        uint32_t acc[2][32];
-        tmem_ld32(lane_base + nl0, acc[0]);
-        tmem_ld32(lane_base + nl0 + 32, acc[1]);
         tmem_ld_wait();
-        if (pc == kEpiCols / 64 - 1) {
+        if (pc + 1 < kEpiCols / 64) {
+          tmem_ld32(lane_base + nl0 + 64, acc[(pc + 1) & 1][0]);
+          tmem_ld32(lane_base + nl0 + 96, acc[(pc + 1) & 1][1]);
+        } else {
+          // Every TMEM load of this warp has completed: release the accumulator.
           tc_fence_before_sync();
           __syncwarp();
           if (lane == 0) mbar_arrive_on(smem_u32(acc_free), 0u);
@@ -354,13 +372,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int nl = nl0 + 32 * u;
+          const uint32_t* a = acc[pc & 1][u];
           uint32_t o[16];
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const float4 a4 = reinterpret_cast<const float4*>(alpha_w)[(nl >> 2) + c];
-            o[2 * c] = pack_bf16x2(a4.x * __uint_as_float(acc[u][4 * c + 0]), a4.y * __uint_as_float(acc[u][4 * c + 1]));
-            o[2 * c + 1] =
-                pack_bf16x2(a4.z * __uint_as_float(acc[u][4 * c + 2]), a4.w * __uint_as_float(acc[u][4 * c + 3]));
+            const uint64_t lo =
+                mul_f32x2(pack_f32x2(a4.x, a4.y), pack_f32x2(__uint_as_float(a[4 * c]), __uint_as_float(a[4 * c + 1])));
+            const uint64_t hi = mul_f32x2(pack_f32x2(a4.z, a4.w),
+                                          pack_f32x2(__uint_as_float(a[4 * c + 2]), __uint_as_float(a[4 * c + 3])));
+            o[2 * c] = pack_bf16x2(__uint_as_float((uint32_t)lo), __uint_as_float((uint32_t)(lo >> 32)));
+            o[2 * c + 1] = pack_bf16x2(__uint_as_float((uint32_t)hi), __uint_as_float((uint32_t)(hi >> 32)));
           }
           if (p.y_mode == 3) {
             uint4* rowp = reinterpret_cast<uint4*>(box + lane * 128);
