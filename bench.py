@@ -79,9 +79,12 @@ def measured_traffic(workload, kernel):
 
 
 def gemm_variant(ck):
-    """Which GEMM kernel the library picks for this layer (the same rule it applies at create time)."""
+    """Which GEMM kernel the library picks for this layer (the rules it applies)."""
     if os.environ.get("SVDQ_GEMM_TILE_N") == "128" or ck.R > 32:
         return "gemm_nvfp4_lr_kernel, 128x128 tiles"
+    if ck.M > 128 and not os.environ.get("SVDQ_GEMM_PAIR", "").startswith("0"):
+        return ("gemm_nvfp4_pair_kernel, 256x256 tiles on 2-CTA clusters (tcgen05 cta_group::2), "
+                "alpha folded into proj_up")
     return "gemm_nvfp4_n256_kernel, 128x256 tiles, alpha folded into proj_up"
 
 

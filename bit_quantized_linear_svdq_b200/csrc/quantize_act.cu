@@ -14,11 +14,14 @@
 // Work decomposition.  A CTA owns 128 token rows and a contiguous slice of
 // K; the K slices of one row tile form a thread-block cluster that reduces
 // its partial L in distributed shared memory (fixed order, deterministic).
-// Inside a CTA (320 threads; two CTAs per SM without rotation):
+// Inside a CTA (320 threads, one CTA per SM):
 //   warp 8 lane 0   TMA producer: x chunk (128 rows x 128 K, two 128B-swizzled
 //                   boxes), proj_down^T chunk (R x 128) and the smooth factors
-//                   into a 2-deep ring; warp 8 also owns the TMEM allocation.
-//   warps 0-7       two threads per row, 64 K elements each: smooth (+ rotate),
+//                   into a ring of up to 4 stages; warp 8 also owns the TMEM
+//                   allocation.
+//   warps 0-7       without rotation: each thread one 16-channel block of four
+//                   rows; with rotation: four threads per row (32 K elements
+//                   each, two rows per chunk in turn): smooth (+ rotate),
 //                   quantize, write codes/scales to global, and write bf16(x_hat)
 //                   back in place over x in shared memory -- exactly the
 //                   128B-swizzled K-major layout the tensor core reads as A.
@@ -54,20 +57,22 @@ constexpr int kXStageBytes = kRows * kChunk * 2;   // 32 KB: two 64-wide swizzle
 constexpr int kXBoxBytes = kXStageBytes / 2;       // 16 KB
 constexpr int kLamStageBytes = kChunk * 8;         // float4 {-s0,-s1,1/s0,1/s1} per channel pair
 // Forward-layout outputs of one chunk are staged in shared memory and written
-// with one TMA tensor store (codes, 128 rows x 64 bytes) and bulk copies (the
-// chunk's two scale atoms, each to its four replicas).
+// with one TMA tensor store (codes, 128 rows x 64 bytes) and one bulk copy (the
+// chunk's two adjacent scale atoms).
 constexpr int kCodeStageBytes = kRows * kChunk / 2;   // 8 KB
 constexpr int kSfStageBytes = 2 * kSfAtomBytes;       // 1 KB
 // Thread layout: 8 compute warps, then the TMA producer warp and the MMA
 // warp.  The unrotated path gives each thread four rows of one 16-channel
 // block column (measured faster than 16 warps of two rows, which need fewer
-// registers than the four-row chains want); the rotated path gives two
-// threads to each row.
+// registers than the four-row chains want); the rotated path gives four
+// threads to each row, two rows per chunk in turn: with ten warps a thread
+// gets at most 168 registers (each SM sub-partition holds three of the warps),
+// and a 64-value slice of the rotation block per thread spilled.
 template <bool ROT>
 struct QCfg {
   static constexpr int kComputeWarps = 8;
   static constexpr int kComputeThreads = 32 * kComputeWarps;
-  static constexpr int kRowsPerThread = ROT ? 1 : 4;     // unrotated path: rows r0 + (128 / 4) * rr
+  static constexpr int kRowsPerThread = ROT ? 2 : 4;     // unrotated: rows r0 + (128 / 4) * rr; rotated: row4, row4 + 64
   static constexpr int kProducerWarp = kComputeWarps, kMmaWarp = kComputeWarps + 1;
   static constexpr int kThreads = 32 * (kComputeWarps + 2);
 };
@@ -241,99 +246,57 @@ __device__ __forceinline__ void write_back_bf16(uint8_t* xs, int row, int c0, co
   *reinterpret_cast<uint4*>(xs + xoff(row, c0 + 1)) = o1;
 }
 
-template <bool TILED>
-__device__ __forceinline__ void store_codes(const QParams& p, int m, int k, const uint32_t (&w)[8]) {
-  // 64 K elements = 32 code bytes of one row, starting at element k.
-  uint8_t* dst = p.codes + (size_t)m * p.codes_pitch + (k >> 1);
-  if (k + 64 <= p.k_limit) {
-    if (TILED) {   // workspace rows are 16-byte aligned
-      reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    } else {       // caller rows are 8-byte aligned (K % 16 == 0)
-      uint2* d = reinterpret_cast<uint2*>(dst);
-      d[0] = make_uint2(w[0], w[1]);
-      d[1] = make_uint2(w[2], w[3]);
-      d[2] = make_uint2(w[4], w[5]);
-      d[3] = make_uint2(w[6], w[7]);
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (k + 16 * j < p.k_limit) reinterpret_cast<uint2*>(dst)[j] = make_uint2(w[2 * j], w[2 * j + 1]);
-  }
-}
-
-template <bool TILED>
-__device__ __forceinline__ void store_scales(const QParams& p, int m, int row, int k, uint32_t sbytes) {
-  // four scale bytes (16-element blocks k/16 .. k/16+3), byte j for block j
-  if (TILED) {
-    uint8_t* atom = p.scales + ((size_t)(m >> 7) * p.ka_pad + (k >> 6)) * kSfAtomBytes + sf_atom_offset(row, 0);
-    *reinterpret_cast<uint32_t*>(atom) = sbytes;
-  } else {
-    uint8_t* dst = p.scales + (size_t)m * p.scales_pitch + (k >> 4);
-    if (k + 64 <= p.k_limit && ((reinterpret_cast<uintptr_t>(dst) & 3u) == 0)) {
-      *reinterpret_cast<uint32_t*>(dst) = sbytes;
-    } else {
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (k + 16 * j < p.k_limit) dst[j] = (uint8_t)(sbytes >> (8 * j));
-    }
-  }
-}
-
-// Rotated path, one thread: the 64 consecutive K elements (half `q` of the
-// chunk, one 128-element rotation block per row) of row `row`.  Codes and
-// scale bytes are returned in registers and stored after the chunk is handed
-// to the tensor core.
-__device__ __forceinline__ void rotate_half(uint8_t* xs, const float4* lam4, const float2* srec, float y6, int row,
-                                            int q, uint32_t (&cw)[8], uint32_t& sbytes) {
-  // The 32 channel pairs of this half: pair 32q + 4c + i at lam_slot(32q + 4c + i).
-  sbytes = 0;
-  // The row's 128-element rotation block is split over lanes 2r (first 64)
-  // and 2r+1 (last 64) of one warp.  Element e of this half is lane (e & 1)
-  // of v[e >> 1].
-  uint64_t v[32];
+// Rotated path, one thread: the 32 consecutive K elements (quarter `qq` of the
+// chunk) of row `row`; lanes 4r .. 4r+3 of a warp hold the four quarters of one
+// row's 128-element rotation block.  Element e of the quarter is lane (e & 1)
+// of v[e >> 1].  Butterfly stages h = 1 .. 16 stay in registers; h = 32 and 64
+// pair the quarter with the one in lane ^ 1 and lane ^ 2, the lower of the two
+// taking a + b and the upper a - b, each as one fused op (+-mine + other) with
+// a single rounding.  Codes and the two scale bytes are returned in registers.
+__device__ __forceinline__ void rotate_quarter(uint8_t* xs, const float4* lam4, const float2* srec, float y6, int row,
+                                               int qq, uint32_t (&cw)[4], uint32_t& sbytes) {
+  uint64_t v[16];
   float big = 0.0f;
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const uint4 pw = *reinterpret_cast<const uint4*>(xs + xoff(row, 8 * q + c));
+  for (int c = 0; c < 4; ++c) {
+    const uint4 pw = *reinterpret_cast<const uint4*>(xs + xoff(row, 4 * qq + c));
     const uint32_t xin[4] = {pw.x, pw.y, pw.z, pw.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float4 l = lam4[lam_slot(32 * q + 4 * c + i)];
+      const float4 l = lam4[lam_slot(16 * qq + 4 * c + i)];
       v[4 * c + i] = div_rn2(bf16x2_to_f2(xin[i]), pk2(l.x, l.y), pk2(l.z, l.w));
       big = amax_nan(amax_nan(big, lo2(v[4 * c + i])), hi2(v[4 * c + i]));
     }
   }
   if (!(big < 3.0e38f)) {            // overflow / NaN (rare): redo with the divide unit
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const uint4 pw = *reinterpret_cast<const uint4*>(xs + xoff(row, 8 * q + c));
+    for (int c = 0; c < 4; ++c) {
+      const uint4 pw = *reinterpret_cast<const uint4*>(xs + xoff(row, 4 * qq + c));
       const uint32_t xin[4] = {pw.x, pw.y, pw.z, pw.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float4 l = lam4[lam_slot(32 * q + 4 * c + i)];
+        const float4 l = lam4[lam_slot(16 * qq + 4 * c + i)];
         v[4 * c + i] = pk2(__fdiv_rn(__uint_as_float(xin[i] << 16), -l.x),
                            __fdiv_rn(__uint_as_float(xin[i] & 0xFFFF0000u), -l.y));
       }
     }
   }
-  // Butterfly stage h = 1: the pair (2i, 2i+1) is the two lanes of v[i];
-  // regroup two words so each packed op yields two results.
+  // h = 1: the pair (2i, 2i+1) is the two lanes of v[i]; regroup two words so
+  // each packed op yields two results.
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
+  for (int j = 0; j < 8; ++j) {
     const uint64_t a = pk2(lo2(v[2 * j]), lo2(v[2 * j + 1]));
     const uint64_t b = pk2(hi2(v[2 * j]), hi2(v[2 * j + 1]));
     const uint64_t sm = add2(a, b), df = sub2(a, b);
     v[2 * j] = pk2(lo2(sm), lo2(df));
     v[2 * j + 1] = pk2(hi2(sm), hi2(df));
   }
-  // Stages h = 2, 4, 8, 16, 32: pairs of packed words (i, i + h/2).
+  // h = 2, 4, 8, 16: words (i, i + h/2).
 #pragma unroll
-  for (int st = 0; st < 5; ++st) {
+  for (int st = 0; st < 4; ++st) {
     const int hp = 1 << st;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < 16; ++i) {
       if ((i & hp) == 0) {
         const uint64_t a = v[i], b = v[i + hp];
         v[i] = add2(a, b);
@@ -341,31 +304,53 @@ __device__ __forceinline__ void rotate_half(uint8_t* xs, const float4* lam4, con
       }
     }
   }
-  // Stage h = 64 across the lane pair: lower half a + b, upper half a - b,
-  // each one fused op (+-mine + other) with a single rounding.
-  {
-    const float sg = q ? -1.0f : 1.0f;
+  // h = 32 (lane ^ 1) and h = 64 (lane ^ 2).
+#pragma unroll
+  for (int st = 0; st < 2; ++st) {
+    const float sg = (qq >> st) & 1 ? -1.0f : 1.0f;
     const uint64_t sg2 = pk2(sg, sg);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float olo = __shfl_xor_sync(0xFFFFFFFFu, lo2(v[i]), 1);
-      const float ohi = __shfl_xor_sync(0xFFFFFFFFu, hi2(v[i]), 1);
+    for (int i = 0; i < 16; ++i) {
+      const float olo = __shfl_xor_sync(0xFFFFFFFFu, lo2(v[i]), 1 << st);
+      const float ohi = __shfl_xor_sync(0xFFFFFFFFu, hi2(v[i]), 1 << st);
       v[i] = fma2(sg2, v[i], pk2(olo, ohi));
     }
   }
   const float cn = 0.0883883461356163f;        // fp32(1/sqrt(128)) = 0x3DB504F3
   const uint64_t cn2 = pk2(cn, cn);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = mul2(v[i], cn2);
+  for (int i = 0; i < 16; ++i) v[i] = mul2(v[i], cn2);
+  sbytes = 0;
 #pragma unroll
-  for (int b = 0; b < 4; ++b) {
+  for (int b = 0; b < 2; ++b) {
     uint64_t blk[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) blk[i] = v[8 * b + i];
     const uint32_t sb = quantize_any(blk, srec, y6, cw[2 * b], cw[2 * b + 1]);
     sbytes |= sb << (8 * b);
-    write_back_bf16(xs, row, 8 * q + 2 * b, blk);
+    write_back_bf16(xs, row, 4 * qq + 2 * b, blk);
   }
+}
+
+// Stage the codes (16 bytes) and two scale bytes of one rotated quarter.
+__device__ __forceinline__ void stage_quarter(uint8_t* cst, uint8_t* sst, int row, int qq, const uint32_t (&cw)[4],
+                                              uint32_t sbytes) {
+  *reinterpret_cast<uint4*>(cst + row * (kChunk / 2) + qq * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+  *reinterpret_cast<uint16_t*>(sst + (qq >> 1) * kSfAtomBytes + sf_atom_offset(row, 2 * (qq & 1))) =
+      (uint16_t)sbytes;
+}
+
+// Row-major (caller layout) stores of one rotated quarter: 32 K elements from k.
+__device__ __forceinline__ void store_quarter(const QParams& p, int m, int k, const uint32_t (&cw)[4],
+                                              uint32_t sbytes) {
+  uint8_t* dst = p.codes + (size_t)m * p.codes_pitch + (k >> 1);   // rows 8-byte aligned (K % 16 == 0)
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+    if (k + 16 * j < p.k_limit) reinterpret_cast<uint2*>(dst)[j] = make_uint2(cw[2 * j], cw[2 * j + 1]);
+  uint8_t* sd = p.scales + (size_t)m * p.scales_pitch + (k >> 4);
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+    if (k + 16 * j < p.k_limit) sd[j] = (uint8_t)(sbytes >> (8 * j));
 }
 
 // Unrotated path, one thread: the 16-channel block column j = t & 7 of the
@@ -496,15 +481,6 @@ __device__ __forceinline__ void stage_cols(uint8_t* cst, uint8_t* sst, int t,
     *reinterpret_cast<uint2*>(cst + row * (kChunk / 2) + j * 8) = make_uint2(cw[rr][0], cw[rr][1]);
     sst[(j >> 2) * kSfAtomBytes + sf_atom_offset(row, j & 3)] = (uint8_t)sb[rr];
   }
-}
-
-// Stage the chunk's codes and compact scale atoms of the rotated mapping.
-__device__ __forceinline__ void stage_half(uint8_t* cst, uint8_t* sst, int row, int q, const uint32_t (&cw)[8],
-                                           uint32_t sbytes) {
-  uint4* c = reinterpret_cast<uint4*>(cst + row * (kChunk / 2) + q * 32);
-  c[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-  c[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-  *reinterpret_cast<uint32_t*>(sst + q * kSfAtomBytes + sf_atom_offset(row, 0)) = sbytes;
 }
 
 template <bool TILED>
@@ -657,7 +633,7 @@ __global__ void __launch_bounds__(QCfg<ROT>::kThreads, 1)
   } else {
     // compute warps: the chunk's 128 rows x 128 channels
     const float y6 = __frcp_rn(6.0f);
-    const int row2 = tid >> 1, q = tid & 1;      // rotated mapping: two threads per row
+    const int row4 = tid >> 2, qq = tid & 3;     // rotated mapping: four threads per row, rows row4 and row4 + 64
     const int nvalid = p.M - m0;                 // rows of this tile that exist (>= 1)
     for (int i = 0; i < nch; ++i) {
       const int s = i % p.stages;
@@ -668,18 +644,22 @@ __global__ void __launch_bounds__(QCfg<ROT>::kThreads, 1)
       const int kc = (c_begin + i) * kChunk;
       uint8_t* xs = X + s * kXStageBytes;
       const float4* lam = reinterpret_cast<const float4*>(LAM + s * kLamStageBytes);
-      uint32_t cw8[8], sbytes = 0;                 // rotated mapping
+      uint32_t cwq[2][4], sq[2];                   // rotated mapping
       uint32_t cw[kColRowsPerThread][2], sb[kColRowsPerThread];   // column mapping
       if (ROT) {
-        // rotate_half exchanges values between lane pairs with full-warp
-        // shuffles, so only a whole warp may skip: all 16 of its rows lie
-        // beyond M (rows beyond M that a warp does process are zero-filled
-        // and rotate to zero).
-        if ((row2 & ~15) < nvalid) {
-          rotate_half(xs, lam, tabs->srec, y6, row2, q, cw8, sbytes);
-        } else {                     // no row of this warp exists: zeros staged
+        // rotate_quarter exchanges values between lanes with full-warp
+        // shuffles, so only a whole warp may skip: all 8 of its rows of the
+        // pass lie beyond M (rows beyond M that a warp does process are
+        // zero-filled and rotate to zero).
 #pragma unroll
-          for (int c = 0; c < 8; ++c) cw8[c] = 0u;
+        for (int ps = 0; ps < 2; ++ps) {
+          if ((row4 & ~7) + 64 * ps < nvalid) {
+            rotate_quarter(xs, lam, tabs->srec, y6, row4 + 64 * ps, qq, cwq[ps], sq[ps]);
+          } else {                   // no row of this warp exists: zeros staged
+#pragma unroll
+            for (int c = 0; c < 4; ++c) cwq[ps][c] = 0u;
+            sq[ps] = 0u;
+          }
         }
       } else if (nvalid >= kRows) {
         smooth_cols<NEG>(xs, lam, tabs->srec, y6, tid, cw, sb);
@@ -691,18 +671,20 @@ __global__ void __launch_bounds__(QCfg<ROT>::kThreads, 1)
         // before the stage was released for this chunk's load.
         uint8_t* cst = CST + s * kCodeStageBytes;
         uint8_t* sst = SST + s * kSfStageBytes;
-        if (ROT)
-          stage_half(cst, sst, row2, q, cw8, sbytes);
-        else
+        if (ROT) {
+          stage_quarter(cst, sst, row4, qq, cwq[0], sq[0]);
+          stage_quarter(cst, sst, row4 + 64, qq, cwq[1], sq[1]);
+        } else
           stage_cols(cst, sst, tid, cw, sb);
       }
       fence_proxy_async_smem();                    // x_hat (and staging) -> async proxy
       mbar_arrive(smem_u32(&xready[s]));
       if (!TILED && ROT) {
-        const int m = m0 + row2, k0 = kc + 64 * q;
-        if (m < p.M && k0 < p.k_limit) {
-          store_codes<false>(p, m, k0, cw8);
-          store_scales<false>(p, m, row2, k0, sbytes);
+        const int k0 = kc + 32 * qq;
+#pragma unroll
+        for (int ps = 0; ps < 2; ++ps) {
+          const int m = m0 + row4 + 64 * ps;
+          if (m < p.M && k0 < p.k_limit) store_quarter(p, m, k0, cwq[ps], sq[ps]);
         }
       } else if (!TILED) {
         store_cols<false>(p, m0, tid, kc, cw, sb);
