@@ -53,7 +53,7 @@ namespace {
 
 constexpr int BM = 256, BMC = 128, BN = 256;     // pair tile rows, rows per CTA, tile columns
 constexpr int kKTileBytes = 128;                 // 256 FP4 elements per row per stage
-constexpr int kStages = 4;
+constexpr int kMaxStages = 4;                    // ring depth: 4, or 3 when the rank-R tiles need the room
 constexpr int kAtoms = 4;                        // 64-element scale atoms per stage
 constexpr int kABytes = BMC * kKTileBytes;       // 16 KB: this CTA's activation rows
 constexpr int kBBytes = (BN / 2) * kKTileBytes;  // 16 KB: this CTA's half of the weight rows
@@ -63,7 +63,6 @@ constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;   // 38 K
 constexpr int kSfWarp0 = 2, kSfWarps = 4;
 constexpr int kEpiWarp0 = 6, kEpiWarps = 4;
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
-constexpr int kSfBufs = kStages;
 constexpr int kSfCols = 48;
 constexpr int kEpiCols = BN * 4 / kEpiWarps;     // columns per epilogue warp
 constexpr int kStageOutBytes = 32 * 128;         // per epilogue warp: a 64-column x 32-row bf16 box
@@ -81,7 +80,8 @@ struct PParams {
   int m_tiles;            // 256-row tiles
   int m_tiles128;         // 128-row scale tiles that exist in the workspace
   int n_tiles;            // 256-column tiles
-  int lr_row_bytes;       // bytes per row of the L / proj_up' tiles in shared memory (32 or 64)
+  int lr_row_bytes;       // bytes per row of one L / proj_up' box in shared memory (32, 64 or 128)
+  int lr_boxes;           // boxes of lr_row_bytes / 2 ranks per row (R <= 32: 1; else ceil(R / 64))
   int y_mode;             // 3: through shared-memory boxes and TMA stores (N % 8 == 0); 0: element stores
 };
 
@@ -103,23 +103,26 @@ __device__ __forceinline__ uint64_t sdesc_rows(uint32_t saddr, int row_bytes) {
          ((uint64_t)((8u * (uint32_t)row_bytes) >> 4) << 32) | (1ull << 46) | (layout << 61);
 }
 
+template <int kStages>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                            const __grid_constant__ CUtensorMap tm_l, const __grid_constant__ CUtensorMap tm_pu,
                            const __grid_constant__ CUtensorMap tm_y, const PParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const int lr_half_bytes = BMC * p.lr_row_bytes;
+  constexpr int kSfBufs = kStages;
+  const int lr_box_bytes = BMC * p.lr_row_bytes;                // 128 rows of one box
+  const int lr_half_bytes = p.lr_boxes * lr_box_bytes;          // this CTA's L rows (or proj_up' rows)
   uint8_t* stages = base;
   uint8_t* OUT = stages + kStages * kStageBytes;                // kEpiWarps x 2 x kStageOutBytes
   uint8_t* ALPHA = OUT + kEpiWarps * 2 * kStageOutBytes;        // kEpiWarps x kEpiCols floats
   uint8_t* LRB = ALPHA + kEpiWarps * kEpiCols * 4;              // {L rows, proj_up' half} of this CTA
   uint64_t* bars = reinterpret_cast<uint64_t*>(LRB + 2 * lr_half_bytes);
-  uint64_t* full = bars;                        // [kStages] both CTAs' A/B landed (even CTA)
-  uint64_t* empty = full + kStages;             // [kStages] pair MMAs done reading the stage
-  uint64_t* sf_ld = empty + kStages;            // [kStages] this CTA's scale atoms landed
-  uint64_t* sf_full = sf_ld + kStages;          // [kSfBufs] scales in both TMEMs (even CTA)
-  uint64_t* lr_full = sf_full + kSfBufs;        // [1] both CTAs' L / proj_up' landed (even CTA)
+  uint64_t* full = bars;                        // [stages] both CTAs' A/B landed (even CTA)
+  uint64_t* empty = full + kMaxStages;          // [stages] pair MMAs done reading the stage
+  uint64_t* sf_ld = empty + kMaxStages;         // [stages] this CTA's scale atoms landed
+  uint64_t* sf_full = sf_ld + kMaxStages;       // [stages] scales in both TMEMs (even CTA)
+  uint64_t* lr_full = sf_full + kMaxStages;     // [1] both CTAs' L / proj_up' landed (even CTA)
   uint64_t* lr_free = lr_full + 1;              // [1] rank-R MMAs done reading them
   uint64_t* acc_full = lr_free + 1;             // [1] accumulator ready
   uint64_t* acc_free = acc_full + 1;            // [1] both epilogues done reading (even CTA)
@@ -208,8 +211,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const uint32_t lf = smem_u32(lr_full);
             if (leader) mbar_arrive_expect_tx(lf, (uint32_t)(4 * lr_half_bytes));
-            tma_load_2d_pair(smem_u32(LRB), &tm_l, lf, 0, mrow0);
-            tma_load_2d_pair(smem_u32(LRB + lr_half_bytes), &tm_pu, lf, 0, nrow0);
+            for (int bx = 0; bx < p.lr_boxes; ++bx) {
+              tma_load_2d_pair(smem_u32(LRB + bx * lr_box_bytes), &tm_l, lf, bx * (p.lr_row_bytes / 2), mrow0);
+              tma_load_2d_pair(smem_u32(LRB + lr_half_bytes + bx * lr_box_bytes), &tm_pu, lf,
+                               bx * (p.lr_row_bytes / 2), nrow0);
+            }
             lr_issued = it + 1;
           }
         }
@@ -253,9 +259,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after_sync();
         const uint32_t la = smem_u32(LRB), pa = la + lr_half_bytes;
-        for (int kk = 0; kk < p.R / 16; ++kk)
-          mma_bf16_pair(tmem + kColAcc, sdesc_rows(la + kk * 32, p.lr_row_bytes),
-                        sdesc_rows(pa + kk * 32, p.lr_row_bytes), idesc_lr, 1u);
+        const int per_box = p.lr_row_bytes / 32;           // K = 16 bf16 = 32 bytes per MMA
+        for (int kk = 0; kk < p.R / 16; ++kk) {
+          const int off = (kk / per_box) * lr_box_bytes + (kk % per_box) * 32;
+          mma_bf16_pair(tmem + kColAcc, sdesc_rows(la + off, p.lr_row_bytes), sdesc_rows(pa + off, p.lr_row_bytes),
+                        idesc_lr, 1u);
+        }
         tc_commit_pair(smem_u32(lr_free), kPairMask);
         tc_commit_pair(smem_u32(acc_full), kPairMask);
       }
@@ -440,12 +449,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-size_t pair_smem_bytes(int row_bytes) {
-  return 1024 + (size_t)kStages * kStageBytes + (size_t)kEpiWarps * (2 * kStageOutBytes + kEpiCols * 4) +
-         (size_t)2 * BMC * row_bytes + 256;
+int pair_lr_boxes(int R) { return R <= 32 ? 1 : (R + 63) / 64; }
+
+size_t pair_smem_bytes(int R, int stages) {
+  return 1024 + (size_t)stages * kStageBytes + (size_t)kEpiWarps * (2 * kStageOutBytes + kEpiCols * 4) +
+         (size_t)2 * pair_lr_boxes(R) * BMC * gemm_pair_lr_row_bytes(R) + 256;
 }
 
-// Pairs that can be resident at once (cached per device and shared-memory size).
+// Deepest ring (4, else 3 stages) that fits beside the rank-R tiles.
+int pair_stages(int R) { return pair_smem_bytes(R, kMaxStages) <= 227 * 1024 ? kMaxStages : kMaxStages - 1; }
+
+// Pairs that can be resident at once (cached per device, ring depth and
+// shared-memory size).
+template <int kStages>
 int max_active_pairs(size_t smem) {
   static std::mutex mu;
   static std::map<std::pair<int, size_t>, int> cache;
@@ -456,7 +472,7 @@ int max_active_pairs(size_t smem) {
   auto f = cache.find(key);
   if (f != cache.end()) return f->second;
   int n = 0;
-  if (ensure_smem_limit(gemm_nvfp4_pair_kernel, smem) == cudaSuccess) {
+  if (ensure_smem_limit(gemm_nvfp4_pair_kernel<kStages>, smem) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -468,45 +484,22 @@ int max_active_pairs(size_t smem) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel<kStages>, &cfg) != cudaSuccess) n = 0;
   }
   cudaGetLastError();   // clear a failed query
   cache[key] = n;
   return n;
 }
 
-}  // namespace
-
-bool gemm_pair_available(int R) {
-  return R <= 32 && max_active_pairs(pair_smem_bytes(gemm_n256_lr_row_bytes(R))) > 0;
+int max_active_pairs_for(int R) {
+  const size_t smem = pair_smem_bytes(R, pair_stages(R));
+  return pair_stages(R) == kMaxStages ? max_active_pairs<kMaxStages>(smem) : max_active_pairs<kMaxStages - 1>(smem);
 }
 
-cudaError_t launch_gemm_nvfp4_pair(const GemmLaunch& L, cudaStream_t stream) {
-  if (L.M <= 0) return cudaSuccess;
-  if (L.R > 32) return cudaErrorInvalidValue;
-  const int row_bytes = gemm_n256_lr_row_bytes(L.R);
-  const size_t smem = pair_smem_bytes(row_bytes);
-  if (smem > 227 * 1024) return cudaErrorInvalidValue;
-  cudaError_t e = ensure_smem_limit(gemm_nvfp4_pair_kernel, smem);
+template <int kStages>
+cudaError_t launch_pair(const GemmLaunch& L, const PParams& p, size_t smem, int max_pairs, cudaStream_t stream) {
+  cudaError_t e = ensure_smem_limit(gemm_nvfp4_pair_kernel<kStages>, smem);
   if (e != cudaSuccess) return e;
-  const int max_pairs = max_active_pairs(smem);
-  if (max_pairs <= 0) return cudaErrorInvalidConfiguration;
-  PParams p;
-  p.sfa = L.sfa;
-  p.sfb = L.sfb;
-  p.alpha = L.alpha;
-  p.y = reinterpret_cast<__nv_bfloat16*>(L.y);
-  p.err = L.err;
-  p.M = L.M;
-  p.N = L.N;
-  p.R = L.R;
-  p.k_tiles = L.k_tiles;
-  p.ka_pad = L.ka_pad;
-  p.m_tiles = (L.M + BM - 1) / BM;
-  p.m_tiles128 = (L.M + BMC - 1) / BMC;
-  p.n_tiles = (L.N + BN - 1) / BN;
-  p.lr_row_bytes = row_bytes;
-  p.y_mode = (L.N % 8) == 0 ? 3 : 0;
   const int tiles = p.m_tiles * p.n_tiles;
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
   cudaLaunchConfig_t cfg = {};
@@ -523,7 +516,44 @@ cudaError_t launch_gemm_nvfp4_pair(const GemmLaunch& L, cudaStream_t stream) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_pair_kernel, L.tm_a, L.tm_b, L.tm_l, L.tm_pu, L.tm_y, p);
+  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_pair_kernel<kStages>, L.tm_a, L.tm_b, L.tm_l, L.tm_pu, L.tm_y, p);
+}
+
+}  // namespace
+
+int gemm_pair_lr_row_bytes(int R) { return R <= 16 ? 32 : (R <= 32 ? 64 : 128); }
+
+bool gemm_pair_available(int R) {
+  return R <= 128 && pair_smem_bytes(R, pair_stages(R)) <= 227 * 1024 && max_active_pairs_for(R) > 0;
+}
+
+cudaError_t launch_gemm_nvfp4_pair(const GemmLaunch& L, cudaStream_t stream) {
+  if (L.M <= 0) return cudaSuccess;
+  if (L.R > 128) return cudaErrorInvalidValue;
+  const int stages = pair_stages(L.R);
+  const size_t smem = pair_smem_bytes(L.R, stages);
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  const int max_pairs = max_active_pairs_for(L.R);
+  if (max_pairs <= 0) return cudaErrorInvalidConfiguration;
+  PParams p;
+  p.sfa = L.sfa;
+  p.sfb = L.sfb;
+  p.alpha = L.alpha;
+  p.y = reinterpret_cast<__nv_bfloat16*>(L.y);
+  p.err = L.err;
+  p.M = L.M;
+  p.N = L.N;
+  p.R = L.R;
+  p.k_tiles = L.k_tiles;
+  p.ka_pad = L.ka_pad;
+  p.m_tiles = (L.M + BM - 1) / BM;
+  p.m_tiles128 = (L.M + BMC - 1) / BMC;
+  p.n_tiles = (L.N + BN - 1) / BN;
+  p.lr_row_bytes = gemm_pair_lr_row_bytes(L.R);
+  p.lr_boxes = pair_lr_boxes(L.R);
+  p.y_mode = (L.N % 8) == 0 ? 3 : 0;
+  return stages == kMaxStages ? launch_pair<kMaxStages>(L, p, smem, max_pairs, stream)
+                              : launch_pair<kMaxStages - 1>(L, p, smem, max_pairs, stream);
 }
 
 }  // namespace svdq

@@ -31,6 +31,7 @@ struct svdq_linear {
   bool splitk;            // few rows: split-K GEMM over a cluster (unless SVDQ_SPLITK=0 at create)
   bool pair;              // more than 128 rows: 256 x 256 tiles on CTA pairs (unless SVDQ_GEMM_PAIR=0 at create)
   int lr_row_bytes;       // 128 x 256 GEMM: bytes per row of its L / proj_up' tiles
+  int pair_row_bytes;     // pair GEMM: bytes per row of one L / proj_up' box
   unsigned* err;          // device error word
   // svdq_linear_forward_host: copy streams and events of its row-chunk pipeline.
   cudaStream_t s_in, s_out;
@@ -370,12 +371,14 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
     // environment asks for the 128 x 128 GEMM (SVDQ_GEMM_TILE_N=128).
     const char* env = std::getenv("SVDQ_GEMM_TILE_N");
     const bool force128 = env && std::strcmp(env, "128") == 0;
-    h->n256 = !(bad & 8u) && d->R <= 32 && !force128;
+    const bool foldable = !(bad & 8u) && !force128;
+    h->n256 = foldable && d->R <= 32;
     const char* sk = std::getenv("SVDQ_SPLITK");
     h->splitk = !(sk && sk[0] == '0');
     // 256 x 256 pair tiles (2-CTA clusters) unless SVDQ_GEMM_PAIR=0.
     const char* pr = std::getenv("SVDQ_GEMM_PAIR");
-    h->pair = h->n256 && !(pr && pr[0] == '0');
+    h->pair = foldable && !(pr && pr[0] == '0');
+    h->pair_row_bytes = svdq::gemm_pair_lr_row_bytes(d->R);
     h->lr_row_bytes = svdq::gemm_n256_lr_row_bytes(d->R);
   }
 #undef CREATE_CUDA
@@ -397,8 +400,10 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
     if ((s = make_tmap(&h->tm_pu_fold, h->pu_fold, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d->R, d->N, (uint64_t)d->R * 2,
                        h->lr_row_bytes / 2, 256, lr_swizzle(h->lr_row_bytes))) != SVDQ_OK)
       return fail(s);
+  }
+  if (h->pair) {
     if ((s = make_tmap(&h->tm_pu_fold128, h->pu_fold, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d->R, d->N,
-                       (uint64_t)d->R * 2, h->lr_row_bytes / 2, 128, lr_swizzle(h->lr_row_bytes))) != SVDQ_OK)
+                       (uint64_t)d->R * 2, h->pair_row_bytes / 2, 128, lr_swizzle(h->pair_row_bytes))) != SVDQ_OK)
       return fail(s);
   }
   *out = h;
@@ -534,7 +539,7 @@ svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, 
   if (h->pair && M > 128 && svdq::gemm_pair_available(h->R)) {
     g.tm_b = h->tm_b;
     if ((s = make_tmap(&g.tm_l, ws + w.lr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->R, M, (uint64_t)h->R * 2,
-                       h->lr_row_bytes / 2, 128, lr_swizzle(h->lr_row_bytes))) != SVDQ_OK)
+                       h->pair_row_bytes / 2, 128, lr_swizzle(h->pair_row_bytes))) != SVDQ_OK)
       return s;
     g.tm_pu = h->tm_pu_fold128;
     g.alpha = h->alpha_fold;

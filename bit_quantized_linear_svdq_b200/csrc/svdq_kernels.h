@@ -74,9 +74,12 @@ cudaError_t launch_gemm_nvfp4_n256(const GemmLaunch& p, cudaStream_t stream);
 // pair (cta_group::2) MMAs; alpha folded as for the 128 x 256 kernel.  The
 // GemmLaunch fields then hold:
 //   tm_b   weight codes: box {128, 128} (each CTA loads its half of the tile)
-//   tm_l   L: box {lr_row_bytes / 2, 128}, swizzle of lr_row_bytes
-//   tm_pu  proj_up' (N, R): box {lr_row_bytes / 2, 128}, same swizzle
-// gemm_pair_available: R <= 32 and at least one pair fits on the device.
+//   tm_l   L: box {row_bytes / 2, 128}, swizzle of row_bytes = gemm_pair_lr_row_bytes(R)
+//   tm_pu  proj_up' (N, R): box {row_bytes / 2, 128}, same swizzle
+//   (for R > 32 the L / proj_up' boxes are {64, 128}, 128B swizzle, one per 64 ranks)
+// gemm_pair_lr_row_bytes: bytes per row of one L / proj_up' box (32, 64 or 128).
+// gemm_pair_available: R <= 128 and at least one pair fits on the device.
+int gemm_pair_lr_row_bytes(int R);
 bool gemm_pair_available(int R);
 cudaError_t launch_gemm_nvfp4_pair(const GemmLaunch& p, cudaStream_t stream);
 

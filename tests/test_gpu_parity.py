@@ -276,6 +276,8 @@ def _select_gemm(kernel, monkeypatch):
     (24, 1008, 300, 128, 0),    # few rows: split-K GEMM, ragged N, R = 128
     (2048, 256, 2560, 32, 0),   # more 256 x 256 tiles than CTA pairs: two tiles per pair
     (260, 512, 300, 32, 0),     # pair tiles with N % 8 != 0: element stores instead of TMA
+    (300, 768, 520, 48, 0),     # pair tiles, rank box only partly filled (R = 48 of 64)
+    (520, 512, 384, 96, 128),   # pair tiles with two rank boxes, three stages, rotation
 ])
 @pytest.mark.parametrize("kernel", ["auto", "n256", "n128"])
 def test_ragged_shapes(M, K, N, R, rot, kernel, monkeypatch):
