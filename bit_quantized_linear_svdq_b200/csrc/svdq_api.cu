@@ -30,6 +30,7 @@ struct svdq_linear {
   bool n256;              // GEMM on 128 x 256 tiles with alpha folded into proj_up
   bool splitk;            // few rows: split-K GEMM over a cluster (unless SVDQ_SPLITK=0 at create)
   bool pair;              // more than 128 rows: 256 x 256 tiles on CTA pairs (unless SVDQ_GEMM_PAIR=0 at create)
+  bool narrow;            // 9..32 rows: y^T on 128-column full-K tiles (unless SVDQ_GEMM_NARROW=0 at create)
   int lr_row_bytes;       // 128 x 256 GEMM: bytes per row of its L / proj_up' tiles
   int pair_row_bytes;     // pair GEMM: bytes per row of one L / proj_up' box
   unsigned* err;          // device error word
@@ -37,7 +38,7 @@ struct svdq_linear {
   cudaStream_t s_in, s_out;
   cudaEvent_t ev_start, ev_out, ev_in[16], ev_comp[16];
   CUtensorMap tm_b, tm_pdT, tm_pu;
-  CUtensorMap tm_b256, tm_pu_fold, tm_pu_fold128;
+  CUtensorMap tm_b256, tm_pu_fold, tm_pu_fold128, tm_pu_fold_n128;
 };
 
 namespace {
@@ -378,6 +379,8 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
     // 256 x 256 pair tiles (2-CTA clusters) unless SVDQ_GEMM_PAIR=0.
     const char* pr = std::getenv("SVDQ_GEMM_PAIR");
     h->pair = foldable && !(pr && pr[0] == '0');
+    const char* nw = std::getenv("SVDQ_GEMM_NARROW");
+    h->narrow = h->n256 && !(nw && nw[0] == '0');
     h->pair_row_bytes = svdq::gemm_pair_lr_row_bytes(d->R);
     h->lr_row_bytes = svdq::gemm_n256_lr_row_bytes(d->R);
   }
@@ -399,6 +402,12 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
   if (h->n256) {
     if ((s = make_tmap(&h->tm_pu_fold, h->pu_fold, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d->R, d->N, (uint64_t)d->R * 2,
                        h->lr_row_bytes / 2, 256, lr_swizzle(h->lr_row_bytes))) != SVDQ_OK)
+      return fail(s);
+  }
+  if (h->narrow) {
+    // 128-row proj_up' boxes: the few-row kernel's rank-R A operand.
+    if ((s = make_tmap(&h->tm_pu_fold_n128, h->pu_fold, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d->R, d->N,
+                       (uint64_t)d->R * 2, h->lr_row_bytes / 2, 128, lr_swizzle(h->lr_row_bytes))) != SVDQ_OK)
       return fail(s);
   }
   if (h->pair) {
@@ -527,6 +536,21 @@ svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, 
   g.R = h->R;
   g.k_tiles = h->k_tiles;
   g.ka_pad = h->ka_pad;
+  // 9..32 rows (R <= 32): y^T on 128-column tiles over the whole of K.
+  if (h->narrow && svdq::gemm_narrow_applies(M, h->R)) {
+    if ((s = make_tmap(&g.tm_a, ws + w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->Kp / 2, M, h->Kp / 2, 128, 32)) !=
+        SVDQ_OK)
+      return s;
+    g.tm_b = h->tm_b;
+    if ((s = make_tmap(&g.tm_l, ws + w.lr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->R, M, (uint64_t)h->R * 2,
+                       h->lr_row_bytes / 2, 32, lr_swizzle(h->lr_row_bytes))) != SVDQ_OK)
+      return s;
+    g.tm_pu = h->tm_pu_fold_n128;
+    g.alpha = h->alpha_fold;
+    cudaError_t e = svdq::launch_gemm_nvfp4_narrow(g, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+    return SVDQ_OK;
+  }
   // Few rows: split K over a cluster so the weight read is spread over the GPU.
   const int S = h->splitk ? svdq::gemm_splitk_slices(M, h->N, h->R, h->k_tiles, num_sms()) : 1;
   if (S > 1) {

@@ -70,6 +70,17 @@ cudaError_t launch_gemm_nvfp4_splitk(const GemmLaunch& p, const void* lowrank, c
                                      cudaStream_t stream);
 cudaError_t launch_gemm_nvfp4_n256(const GemmLaunch& p, cudaStream_t stream);
 
+// The same product for 9..32 rows (R <= 32, alpha folded), computed as
+// y^T: 128 output columns (weight rows, the MMA's M) by the token rows (N =
+// 32) over the whole of K per CTA (persistent), no cross-CTA sums.
+// GemmLaunch fields:
+//   tm_a   activation codes: box {128, 32} (rows 0..31)
+//   tm_b   weight codes: box {128, 128}
+//   tm_l   L: box {lr_row_bytes / 2, 32}, swizzle of lr_row_bytes
+//   tm_pu  proj_up' (N, R): box {lr_row_bytes / 2, 128}, same swizzle
+bool gemm_narrow_applies(int M, int R);
+cudaError_t launch_gemm_nvfp4_narrow(const GemmLaunch& p, cudaStream_t stream);
+
 // The same product on 256 x 256 tiles, each computed by a 2-CTA cluster with
 // pair (cta_group::2) MMAs; alpha folded as for the 128 x 256 kernel.  The
 // GemmLaunch fields then hold:

@@ -253,10 +253,14 @@ def test_full_workload_parity(name):
 # ------------------------------------------------------------------ ragged shapes and edge cases
 
 def _select_gemm(kernel, monkeypatch):
-    """"auto": the library's choice (split-K over a cluster for few rows, else
-    with alpha folded when R <= 32: 256 x 256 tiles on CTA pairs above 128
-    rows, 128 x 256 tiles otherwise; else 128 x 128); "n256" / "n128": the
-    one-CTA persistent kernels without split-K."""
+    """"auto": the library's choice (alpha folded: 9..32 rows with R <= 32 ->
+    y^T on 128-column full-K tiles; above 128 rows -> 256 x 256 tiles on CTA pairs;
+    otherwise split-K over a cluster for at most 32 rows, 128 x 256 tiles for
+    R <= 32, 128 x 128 tiles); "splitk": the same without the y^T kernel,
+    so split-K serves every few-row shape; "n256" / "n128": the one-CTA
+    persistent kernels alone."""
+    if kernel in ("splitk", "n256", "n128"):
+        monkeypatch.setenv("SVDQ_GEMM_NARROW", "0")
     if kernel in ("n256", "n128"):
         monkeypatch.setenv("SVDQ_SPLITK", "0")
         monkeypatch.setenv("SVDQ_GEMM_PAIR", "0")
@@ -278,8 +282,10 @@ def _select_gemm(kernel, monkeypatch):
     (260, 512, 300, 32, 0),     # pair tiles with N % 8 != 0: element stores instead of TMA
     (300, 768, 520, 48, 0),     # pair tiles, rank box only partly filled (R = 48 of 64)
     (520, 512, 384, 96, 128),   # pair tiles with two rank boxes, three stages, rotation
+    (20, 512, 300, 32, 0),      # 9..32 rows: y^T on 128-column tiles, ragged N
+    (29, 768, 136, 16, 128),    # the same with rotation, R = 16
 ])
-@pytest.mark.parametrize("kernel", ["auto", "n256", "n128"])
+@pytest.mark.parametrize("kernel", ["auto", "splitk", "n256", "n128"])
 def test_ragged_shapes(M, K, N, R, rot, kernel, monkeypatch):
     """Every GEMM kernel on every ragged shape (see _select_gemm)."""
     _select_gemm(kernel, monkeypatch)
@@ -291,7 +297,7 @@ def test_ragged_shapes(M, K, N, R, rot, kernel, monkeypatch):
     check_forward(layer, ck)
 
 
-@pytest.mark.parametrize("kernel", ["auto", "n256", "n128"])
+@pytest.mark.parametrize("kernel", ["auto", "splitk", "n256", "n128"])
 def test_zero_alpha_columns(kernel, monkeypatch):
     """Columns with wcscales = 0 reduce to the rank-R branch alone, in every
     GEMM kernel (the folded one gives them alpha' = 1 and zero weight scales)."""
