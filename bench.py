@@ -325,6 +325,32 @@ def run_ours(args, world, rank, local):
     t_gemm = timed(g_gemm)
     t_full_max = max_over_ranks(world, t_full)
 
+    # The offline weight quantizer (svdq_quantize_weight) on this layer's
+    # weight shape: seeded dense bf16 W ~ N(0, 0.02), one per replica set.
+    gen = torch.Generator(device="cuda").manual_seed(7)
+    wsets = []
+    for i in range(N_SETS):
+        w = (torch.randn((N, K), generator=gen, device="cuda") * 0.02).to(torch.bfloat16)
+        wsets.append((w, torch.empty((N, K // 2), dtype=torch.uint8, device="cuda"),
+                      torch.empty((K // 16, N), dtype=torch.uint8, device="cuda")))
+
+    def wq(i):
+        w, qw, wsc = wsets[i % N_SETS]
+        S.svdq_quantize_weight(w.data_ptr(), N, K, ck.rotate_block, qw.data_ptr(), wsc.data_ptr(), stream)
+
+    g_wq = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        for i in range(N_SETS):
+            wq(i)
+        stream.synchronize()
+        with torch.cuda.graph(g_wq, stream=stream):
+            for i in range(args.steps):
+                wq(i)
+        g_wq.replay()
+    torch.cuda.synchronize()
+    t_wq = timed(g_wq)
+    del g_wq, wsets
+
     # End-to-end through the host-buffer C ABI call: H2D of x, forward, D2H of y, sync.
     layer, x, y, ws = sets[0]
     xh = x.cpu().pin_memory()
@@ -354,12 +380,18 @@ def run_ours(args, world, rank, local):
     fp4_peak = pk["bf16_tflops"] * FP4_PER_BF16
     us_q = t_quant / args.steps * 1e6
     us_g = t_gemm / args.steps * 1e6
+    us_wq = t_wq / args.steps * 1e6
+    wq_bytes = 2.0 * N * K + N * K / 2 + N * K / 16
     q_gbs = quant_bytes(M, K, R) / (us_q * 1e-6) / 1e9
     g_flops = 2.0 * M * N * K + 2.0 * M * N * R
     g_tf = g_flops / (us_g * 1e-6) / 1e12
     kernels = {
         "quantize_act": {"us": us_q, "bound": "hbm", "algorithmic_bytes": quant_bytes(M, K, R),
                          "achieved_gbs": q_gbs, "frac_of_hbm": q_gbs / pk["hbm_gbs"]},
+        "quantize_weight": {"us": us_wq, "bound": "hbm", "algorithmic_bytes": wq_bytes,
+                            "achieved_gbs": wq_bytes / (us_wq * 1e-6) / 1e9,
+                            "frac_of_hbm": wq_bytes / (us_wq * 1e-6) / 1e9 / pk["hbm_gbs"],
+                            "note": "offline step (dense weight -> NVFP4), on this layer's weight shape"},
         "gemm_nvfp4": {"us": us_g, "bound": "tensor", "variant": gemm_variant(ck), "algorithmic_flops": g_flops,
                        "achieved_tflops": g_tf, "frac_of_fp4": g_tf / fp4_peak,
                        "algorithmic_bytes": gemm_bytes(M, K, N, R),

@@ -23,7 +23,7 @@ __all__ = [
     "svdq_linear_create", "svdq_linear_destroy", "svdq_workspace_bytes", "svdq_quantize_act",
     "svdq_linear_forward", "svdq_linear_forward_host", "svdq_linear_forward_quantize",
     "svdq_linear_forward_gemm", "svdq_device_status", "svdq_status_string",
-    "svdq_last_error", "svdq_version", "SVDQLinear", "STATUS",
+    "svdq_last_error", "svdq_version", "svdq_quantize_weight", "quantize_weight", "SVDQLinear", "STATUS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -90,6 +90,7 @@ def load_library() -> ctypes.CDLL:
         "svdq_status_string": (ctypes.c_char_p, [ci]),
         "svdq_last_error": (ctypes.c_char_p, []),
         "svdq_version": (ci, []),
+        "svdq_quantize_weight": (ci, [vp, ci, ci, ci, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -189,6 +190,11 @@ def svdq_linear_forward_noalloc(handle, x_ptr, M, y_ptr, stream=None) -> None:
     _check(st, "svdq_linear_forward_noalloc")
 
 
+def svdq_quantize_weight(w_ptr, N, K, rotate_block, qweight_ptr, wscales_ptr, stream=None) -> None:
+    _check(load_library().svdq_quantize_weight(w_ptr, N, K, rotate_block, qweight_ptr, wscales_ptr,
+                                               _stream(stream)), "svdq_quantize_weight")
+
+
 def svdq_device_status(handle) -> int:
     flags = ctypes.c_int(0)
     st = load_library().svdq_device_status(handle, ctypes.byref(flags))
@@ -206,6 +212,19 @@ def _need(t: torch.Tensor, name: str, dtype, shape) -> None:
         raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
     if not t.is_cuda or not t.is_contiguous():
         raise ValueError(f"{name}: must be a contiguous CUDA tensor")
+
+
+def quantize_weight(w: torch.Tensor, rotate_block: int = 0, stream=None):
+    """Dense bf16 W (N, K) on the GPU -> (qweight (N, K/2) uint8, wscales (K/16, N) uint8),
+    the checkpoint's weight tensors (optional 128-block row rotation)."""
+    if w.dim() != 2:
+        raise ValueError("w must be (N, K)")
+    N, K = w.shape
+    _need(w, "w", torch.bfloat16, (N, K))
+    qweight = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
+    wscales = torch.empty((K // 16, N), dtype=torch.uint8, device=w.device)
+    svdq_quantize_weight(w.data_ptr(), N, K, rotate_block, qweight.data_ptr(), wscales.data_ptr(), stream)
+    return qweight, wscales
 
 
 class SVDQLinear:

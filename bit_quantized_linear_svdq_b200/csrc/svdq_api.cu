@@ -598,6 +598,18 @@ svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, 
 
 }  // namespace
 
+svdq_status svdq_quantize_weight(const void* w, int N, int K, int rotate_block, void* qweight, void* wscales,
+                                 void* stream) {
+  if (!w || !qweight || !wscales || !aligned16(w) || (reinterpret_cast<uintptr_t>(qweight) & 7u) != 0)
+    return SVDQ_ERR_INVALID_ARG;
+  if (N < 1 || K < 16 || K % 16 != 0) return SVDQ_ERR_SHAPE;
+  if (rotate_block != 0 && (rotate_block != 128 || K % 128 != 0)) return SVDQ_ERR_SHAPE;
+  cudaError_t e = svdq::launch_quantize_weight(w, N, K, rotate_block, qweight, wscales,
+                                               static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "quantize_weight launch");
+  return SVDQ_OK;
+}
+
 svdq_status svdq_linear_forward_quantize(const svdq_linear* h, const void* x, int M, void* workspace, void* stream) {
   svdq_status s = check_forward_args(h, M, workspace);
   if (s != SVDQ_OK || M == 0) return s;

@@ -31,6 +31,11 @@ struct QuantLaunch {
 };
 cudaError_t launch_quantize_act(const QuantLaunch& p, cudaStream_t stream);
 
+// Offline NVFP4 quantization of a dense bf16 weight (N, K) -> qweight (N, K/2),
+// wscales (K/16, N), optional 128-block row rotation.
+cudaError_t launch_quantize_weight(const void* w, int N, int K, int rotate_block, void* qweight, void* wscales,
+                                   cudaStream_t stream);
+
 // Block-scaled NVFP4 GEMM with the rank-R up-projection and the
 // wcscales * wtscale scaling fused into the epilogue.
 struct GemmLaunch {

@@ -182,6 +182,25 @@ SVDQ_API svdq_status svdq_linear_forward_noalloc(const svdq_linear* h, const voi
                                                  void* stream);
 
 /*
+ * svdq_quantize_weight -- offline NVFP4 quantization of a dense weight on the
+ * GPU (the checkpoint's weight tensors from a bf16 W), with the optional
+ * rotation of every row by blockdiag(H_128 / sqrt(128)) ("Rotate in
+ * quantization and its vLLM implementation", section 2.1: the offline W' = R W,
+ * which in the checkpoint's (N, K) orientation rotates each row like an
+ * activation row).  Same rules as the activation quantizer: fp32 butterfly,
+ * scale = e4m3_rne_satfinite(fp32(amax/6)), code = e2m1_rne_satfinite(fp32(w/scale)).
+ *   w        (N, K)    bf16 in, 16-byte aligned
+ *   qweight  (N, K/2)  uint8 out: packed E2M1, element 2j in the low nibble of byte j; 8-byte aligned
+ *   wscales  (K/16, N) uint8 out: e4m3 scale bytes, wscales[k/16, n] scales w[n, k]
+ * K must be a positive multiple of 16 (of 128 when rotate_block == 128), N >= 1,
+ * rotate_block 0 or 128 (else SVDQ_ERR_SHAPE).  Caller-owned device buffers;
+ * asynchronous on `stream`.  The outputs are svdq_linear_desc's qweight and
+ * wscales.
+ */
+SVDQ_API svdq_status svdq_quantize_weight(const void* w, int N, int K, int rotate_block, void* qweight,
+                                          void* wscales, void* stream);
+
+/*
  * svdq_device_status -- synchronize the handle's device and read + clear its
  * device error word (nonzero when a kernel's bounded wait expired: the kernel
  * then skipped its remaining work, released its tensor memory and returned).

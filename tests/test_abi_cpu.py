@@ -21,7 +21,7 @@ def test_exports_every_declared_symbol(lib):
         "svdq_linear_create", "svdq_linear_destroy", "svdq_workspace_bytes", "svdq_quantize_act",
         "svdq_linear_forward", "svdq_linear_forward_host", "svdq_device_status", "svdq_status_string",
         "svdq_last_error", "svdq_version", "svdq_linear_forward_quantize", "svdq_linear_forward_gemm",
-        "svdq_linear_forward_noalloc"}
+        "svdq_linear_forward_noalloc", "svdq_quantize_weight"}
     for n in names:
         assert hasattr(lib, n), n
 
@@ -74,3 +74,20 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(S, "library_path", lambda: str(tmp_path / "nope.so"))
     with pytest.raises(RuntimeError, match="not built"):
         S.load_library()
+
+
+@pytest.mark.parametrize("args,status", [
+    ((0, 16, 256, 0, 16, 16), 1),        # null weight
+    ((16, 16, 256, 0, 0, 16), 1),        # null qweight
+    ((16, 16, 256, 0, 16, 0), 1),        # null wscales
+    ((8, 16, 256, 0, 16, 16), 1),        # weight not 16-byte aligned
+    ((16, 16, 256, 0, 12, 16), 1),       # qweight not 8-byte aligned
+    ((16, 16, 24, 0, 16, 16), 2),        # K % 16
+    ((16, 0, 256, 0, 16, 16), 2),        # N < 1
+    ((16, 16, 272, 128, 16, 16), 2),     # rotation block does not divide K
+    ((16, 16, 256, 64, 16, 16), 2),      # rotation block other than 128
+])
+def test_quantize_weight_argument_errors(lib, args, status):
+    """Argument errors are answered on the host, before any launch."""
+    w, N, K, rot, qw, ws = args
+    assert lib.svdq_quantize_weight(w, N, K, rot, qw, ws, None) == status
