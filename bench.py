@@ -338,18 +338,33 @@ def run_ours(args, world, rank, local):
         w, qw, wsc = wsets[i % N_SETS]
         S.svdq_quantize_weight(w.data_ptr(), N, K, ck.rotate_block, qw.data_ptr(), wsc.data_ptr(), stream)
 
-    g_wq = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        for i in range(N_SETS):
-            wq(i)
-        stream.synchronize()
-        with torch.cuda.graph(g_wq, stream=stream):
-            for i in range(args.steps):
-                wq(i)
-        g_wq.replay()
-    torch.cuda.synchronize()
+    def graph_calls(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            for i in range(N_SETS):
+                fn(i)
+            stream.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(args.steps):
+                    fn(i)
+            g.replay()
+        torch.cuda.synchronize()
+        return g
+
+    g_wq = graph_calls(wq)
     t_wq = timed(g_wq)
     del g_wq, wsets
+
+    # The standalone Hadamard transform, in place on M rows of 4096 bf16.
+    HN = 4096
+    hsets = [torch.randn((M, HN), generator=gen, device="cuda").to(torch.bfloat16) for _ in range(N_SETS)]
+
+    def ht(i):
+        S.svdq_hadamard_transform(hsets[i % N_SETS].data_ptr(), M, HN, 0, stream)
+
+    g_ht = graph_calls(ht)
+    t_ht = timed(g_ht)
+    del g_ht, hsets
 
     # End-to-end through the host-buffer C ABI call: H2D of x, forward, D2H of y, sync.
     layer, x, y, ws = sets[0]
@@ -381,6 +396,8 @@ def run_ours(args, world, rank, local):
     us_q = t_quant / args.steps * 1e6
     us_g = t_gemm / args.steps * 1e6
     us_wq = t_wq / args.steps * 1e6
+    us_ht = t_ht / args.steps * 1e6
+    ht_bytes = 2.0 * 2 * M * HN
     wq_bytes = 2.0 * N * K + N * K / 2 + N * K / 16
     q_gbs = quant_bytes(M, K, R) / (us_q * 1e-6) / 1e9
     g_flops = 2.0 * M * N * K + 2.0 * M * N * R
@@ -392,6 +409,10 @@ def run_ours(args, world, rank, local):
                             "achieved_gbs": wq_bytes / (us_wq * 1e-6) / 1e9,
                             "frac_of_hbm": wq_bytes / (us_wq * 1e-6) / 1e9 / pk["hbm_gbs"],
                             "note": "offline step (dense weight -> NVFP4), on this layer's weight shape"},
+        "hadamard_transform": {"us": us_ht, "bound": "hbm", "algorithmic_bytes": ht_bytes,
+                               "achieved_gbs": ht_bytes / (us_ht * 1e-6) / 1e9,
+                               "frac_of_hbm": ht_bytes / (us_ht * 1e-6) / 1e9 / pk["hbm_gbs"],
+                               "note": f"standalone transform, in place on {M} x {HN} bf16"},
         "gemm_nvfp4": {"us": us_g, "bound": "tensor", "variant": gemm_variant(ck), "algorithmic_flops": g_flops,
                        "achieved_tflops": g_tf, "frac_of_fp4": g_tf / fp4_peak,
                        "algorithmic_bytes": gemm_bytes(M, K, N, R),

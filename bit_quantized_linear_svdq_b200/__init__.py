@@ -23,7 +23,7 @@ __all__ = [
     "svdq_linear_create", "svdq_linear_destroy", "svdq_workspace_bytes", "svdq_quantize_act",
     "svdq_linear_forward", "svdq_linear_forward_host", "svdq_linear_forward_quantize",
     "svdq_linear_forward_gemm", "svdq_device_status", "svdq_status_string",
-    "svdq_last_error", "svdq_version", "svdq_quantize_weight", "quantize_weight", "SVDQLinear", "STATUS",
+    "svdq_last_error", "svdq_version", "svdq_quantize_weight", "quantize_weight", "svdq_hadamard_transform", "hadamard_transform", "SVDQLinear", "STATUS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -91,6 +91,7 @@ def load_library() -> ctypes.CDLL:
         "svdq_last_error": (ctypes.c_char_p, []),
         "svdq_version": (ci, []),
         "svdq_quantize_weight": (ci, [vp, ci, ci, ci, vp, vp, vp]),
+        "svdq_hadamard_transform": (ci, [vp, ci, ci, ci, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -193,6 +194,23 @@ def svdq_linear_forward_noalloc(handle, x_ptr, M, y_ptr, stream=None) -> None:
 def svdq_quantize_weight(w_ptr, N, K, rotate_block, qweight_ptr, wscales_ptr, stream=None) -> None:
     _check(load_library().svdq_quantize_weight(w_ptr, N, K, rotate_block, qweight_ptr, wscales_ptr,
                                                _stream(stream)), "svdq_quantize_weight")
+
+
+def svdq_hadamard_transform(x_ptr, rows, n, dtype, stream=None) -> None:
+    _check(load_library().svdq_hadamard_transform(x_ptr, rows, n, dtype, _stream(stream)), "svdq_hadamard_transform")
+
+
+def hadamard_transform(x: torch.Tensor, inplace: bool = True, stream=None) -> torch.Tensor:
+    """x <- x H_n / sqrt(n) along the last dimension (n a power of two <= 32768), bf16 or fp16."""
+    if x.dtype not in (torch.bfloat16, torch.float16):
+        raise TypeError("x must be bf16 or fp16")
+    if not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA tensor")
+    y = x if inplace else x.clone()
+    n = y.shape[-1] if y.dim() else 1
+    rows = y.numel() // n if n else 0
+    svdq_hadamard_transform(y.data_ptr(), rows, n, 0 if y.dtype == torch.bfloat16 else 1, stream)
+    return y
 
 
 def svdq_device_status(handle) -> int:

@@ -598,6 +598,18 @@ svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, 
 
 }  // namespace
 
+svdq_status svdq_hadamard_transform(void* x, int rows, int n, int dtype, void* stream) {
+  if (rows < 0 || (dtype != 0 && dtype != 1)) return SVDQ_ERR_INVALID_ARG;
+  if (n < 1 || n > 32768 || (n & (n - 1)) != 0) return SVDQ_ERR_SHAPE;
+  if (rows == 0) return SVDQ_OK;
+  if (!x || (reinterpret_cast<uintptr_t>(x) & 1u) != 0) return SVDQ_ERR_INVALID_ARG;
+  int log2n = 0;
+  while ((1 << log2n) < n) ++log2n;
+  cudaError_t e = svdq::launch_hadamard_transform(x, rows, log2n, dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "hadamard_transform launch");
+  return SVDQ_OK;
+}
+
 svdq_status svdq_quantize_weight(const void* w, int N, int K, int rotate_block, void* qweight, void* wscales,
                                  void* stream) {
   if (!w || !qweight || !wscales || !aligned16(w) || (reinterpret_cast<uintptr_t>(qweight) & 7u) != 0)

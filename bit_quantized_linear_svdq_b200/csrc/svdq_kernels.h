@@ -31,6 +31,10 @@ struct QuantLaunch {
 };
 cudaError_t launch_quantize_act(const QuantLaunch& p, cudaStream_t stream);
 
+// Standalone Walsh-Hadamard transform of rows of length 2^log2n (<= 2^15),
+// in place; dtype 0 = bf16, 1 = fp16.
+cudaError_t launch_hadamard_transform(void* x, int rows, int log2n, int dtype, cudaStream_t stream);
+
 // Offline NVFP4 quantization of a dense bf16 weight (N, K) -> qweight (N, K/2),
 // wscales (K/16, N), optional 128-block row rotation.
 cudaError_t launch_quantize_weight(const void* w, int N, int K, int rotate_block, void* qweight, void* wscales,

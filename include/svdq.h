@@ -182,6 +182,22 @@ SVDQ_API svdq_status svdq_linear_forward_noalloc(const svdq_linear* h, const voi
                                                  void* stream);
 
 /*
+ * svdq_hadamard_transform -- the standalone in-place Walsh-Hadamard transform
+ * x <- x H_n / sqrt(n) of every row ("Rotate in quantization and its vLLM
+ * implementation", section 3.1, the Hadacore transform: Sylvester recursion,
+ * no stored matrix; H symmetric, so the operation is its own inverse).
+ *   x      (rows, n) bf16 (dtype 0) or fp16 (dtype 1), row-major, 2-byte aligned,
+ *          transformed in place
+ *   n      power of two, 1 <= n <= 32768 (else SVDQ_ERR_SHAPE)
+ *   rows   >= 0; rows == 0 is a no-op
+ * Arithmetic in fp32: butterfly stages h = 1, 2, ..., n/2 in that order
+ * ((x[i], x[i+h]) -> (x[i] + x[i+h], x[i] - x[i+h]) for i & h == 0), one
+ * multiply by fp32(1/sqrt(n)), then round to nearest even in the storage type.
+ * Caller-owned device memory; asynchronous on `stream`.
+ */
+SVDQ_API svdq_status svdq_hadamard_transform(void* x, int rows, int n, int dtype, void* stream);
+
+/*
  * svdq_quantize_weight -- offline NVFP4 quantization of a dense weight on the
  * GPU (the checkpoint's weight tensors from a bf16 W), with the optional
  * rotation of every row by blockdiag(H_128 / sqrt(128)) ("Rotate in

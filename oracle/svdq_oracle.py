@@ -203,6 +203,40 @@ def rotate_rows_f64(v: np.ndarray, block: int) -> np.ndarray:
     return hadamard_butterfly(np.asarray(v, np.float64), block, np.float64) / np.sqrt(block)
 
 
+def f32_to_bf16_bits(v32: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 bit patterns, round to nearest, ties to even (NaN -> 0x7FC0 with its sign)."""
+    v32 = np.asarray(v32, dtype=np.float32)
+    u = v32.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+    nan = np.isnan(v32)
+    r[nan] = (np.uint16(0x7FC0) | ((u[nan] >> 16) & 0x8000).astype(np.uint16))
+    return r
+
+
+def hadamard_transform(x_bits: np.ndarray, n: int, dtype: str = "bf16") -> np.ndarray:
+    """The standalone Walsh-Hadamard transform of each length-n row (n = 2^k):
+    x <- x H_n / sqrt(n), in fp32 as the online rotation (the butterfly stages
+    h = 1, 2, ..., n/2 in that order, then one multiply by fp32(1/sqrt(n))),
+    rounded to the storage type (round to nearest, ties to even).
+
+    "Rotate in quantization and its vLLM implementation", section 3.1: the
+    Hadacore transform uses the Sylvester recursion with no stored matrix, and
+    since H is symmetric the same operation is its own inverse.  dtype is
+    "bf16" or "fp16"; x_bits are the row-major (rows, n) bit patterns.
+    """
+    x_bits = np.asarray(x_bits, dtype=np.uint16)
+    if dtype == "bf16":
+        x32 = bf16_to_f32(x_bits)
+    elif dtype == "fp16":
+        x32 = x_bits.view(np.float16).astype(np.float32)
+    else:
+        raise ValueError(dtype)
+    r = rotate_rows_fp32(x32, n)
+    if dtype == "bf16":
+        return f32_to_bf16_bits(r)
+    return r.astype(np.float16).view(np.uint16)
+
+
 # ----------------------------------------------------------------------------
 # Activation path
 # ----------------------------------------------------------------------------

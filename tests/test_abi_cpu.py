@@ -21,7 +21,7 @@ def test_exports_every_declared_symbol(lib):
         "svdq_linear_create", "svdq_linear_destroy", "svdq_workspace_bytes", "svdq_quantize_act",
         "svdq_linear_forward", "svdq_linear_forward_host", "svdq_device_status", "svdq_status_string",
         "svdq_last_error", "svdq_version", "svdq_linear_forward_quantize", "svdq_linear_forward_gemm",
-        "svdq_linear_forward_noalloc", "svdq_quantize_weight"}
+        "svdq_linear_forward_noalloc", "svdq_quantize_weight", "svdq_hadamard_transform"}
     for n in names:
         assert hasattr(lib, n), n
 
@@ -91,3 +91,18 @@ def test_quantize_weight_argument_errors(lib, args, status):
     """Argument errors are answered on the host, before any launch."""
     w, N, K, rot, qw, ws = args
     assert lib.svdq_quantize_weight(w, N, K, rot, qw, ws, None) == status
+
+
+@pytest.mark.parametrize("args,status", [
+    ((16, 4, 3, 0), 2),          # n not a power of two
+    ((16, 4, 0, 0), 2),          # n < 1
+    ((16, 4, 65536, 0), 2),      # n > 32768
+    ((16, 4, 64, 2), 1),         # dtype other than bf16 / fp16
+    ((16, -1, 64, 0), 1),        # rows < 0
+    ((0, 4, 64, 0), 1),          # null x
+    ((17, 4, 64, 0), 1),         # x not 2-byte aligned
+    ((0, 0, 64, 0), 0),          # no rows: no-op
+])
+def test_hadamard_transform_argument_errors(lib, args, status):
+    x, rows, n, dt = args
+    assert lib.svdq_hadamard_transform(x, rows, n, dt, None) == status

@@ -464,3 +464,53 @@ def test_rotated_weight_quantizer_roundtrip():
     back = O.rotate_rows_f64(Wq, 128)
     rel = np.linalg.norm(back - O.bf16_to_f32(_bf16_bits(W))) / np.linalg.norm(W)
     assert rel < 0.2          # 4-bit with coarse (subnormal) e4m3 scales
+
+
+# ---------------------------------------------------------------- [rot] section 3.1: the standalone transform
+
+def test_f32_to_bf16_matches_torch():
+    # The library conversion (round to nearest even) on random values, ties,
+    # subnormals, the largest finite values and infinities.
+    rng = np.random.default_rng(11)
+    v = rng.standard_normal(20000).astype(np.float32) * np.float32(3.0) ** rng.integers(-40, 40, 20000)
+    ties = (np.arange(1, 2000, dtype=np.uint32) << 16 | 0x8000).view(np.float32)
+    special = np.array([0.0, -0.0, 1e-40, -1e-40, 3.4e38, -3.4e38, np.inf, -np.inf], dtype=np.float32)
+    allv = np.concatenate([v, ties, -ties, special]).astype(np.float32)
+    ref = torch.from_numpy(allv).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(O.f32_to_bf16_bits(allv), ref)
+    nanbits = O.f32_to_bf16_bits(np.array([np.nan], dtype=np.float32))
+    assert (nanbits[0] & 0x7F80) == 0x7F80 and (nanbits[0] & 0x7F) != 0
+
+
+@pytest.mark.parametrize("n", [1, 2, 8, 64, 512, 2048])
+def test_hadamard_transform_equals_dense(n):
+    # Hadacore's check (section 3.1): the transform equals x @ H^T (normalised),
+    # here within fp32 accumulation error plus one bf16 rounding.
+    rng = np.random.default_rng(n + 1)
+    x = rng.standard_normal((3, n)).astype(np.float32)
+    xb = O.f32_to_bf16_bits(x)
+    y = O.bf16_to_f32(O.hadamard_transform(xb, n)).astype(np.float64)
+    H = O.sylvester_hadamard(n) / np.sqrt(n)
+    dense = O.bf16_to_f32(xb).astype(np.float64) @ H.T
+    tol = 2.0 ** -8 * np.abs(dense) + 1e-6 * np.sqrt(n) * np.abs(dense).max()
+    assert np.all(np.abs(y - dense) <= tol)
+
+
+@pytest.mark.parametrize("n,dtype", [(16, "bf16"), (4096, "bf16"), (32768, "bf16"), (1024, "fp16")])
+def test_hadamard_transform_involution_and_norm(n, dtype):
+    # Applying the transform twice returns x up to the two roundings to the
+    # storage type; one application preserves the row norm (H / sqrt(n) is
+    # orthogonal); large n agrees with the exact fp64 butterfly.
+    rng = np.random.default_rng(n)
+    x = rng.standard_normal((2, n)).astype(np.float32)
+    xb = O.f32_to_bf16_bits(x) if dtype == "bf16" else x.astype(np.float16).view(np.uint16)
+    dec = (lambda b: O.bf16_to_f32(b)) if dtype == "bf16" else (lambda b: b.view(np.float16).astype(np.float32))
+    x0 = dec(xb).astype(np.float64)
+    y = O.hadamard_transform(xb, n, dtype)
+    yy = dec(y).astype(np.float64)
+    exact = O.rotate_rows_f64(x0, n)
+    eps = 2.0 ** -8 if dtype == "bf16" else 2.0 ** -11
+    assert np.max(np.abs(yy - exact)) <= eps * np.abs(exact).max() + 1e-5 * np.abs(exact).max()
+    np.testing.assert_allclose(np.linalg.norm(yy, axis=1), np.linalg.norm(x0, axis=1), rtol=4 * eps)
+    back = dec(O.hadamard_transform(y, n, dtype)).astype(np.float64)
+    assert np.max(np.abs(back - x0)) <= 4 * eps * np.abs(x0).max()
