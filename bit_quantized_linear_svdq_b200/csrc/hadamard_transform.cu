@@ -9,13 +9,14 @@
 // i & h == 0 by (x[i] + x[i+h], x[i] - x[i+h]); then one multiply by
 // fp32(1/sqrt(n)); then round to the storage type (to nearest, ties to even).
 //
-// A CTA holds whole rows in shared memory as fp32 (element i at word
-// i + i/32, so both the 32-element runs of the first pass and the strided
-// groups of the later ones hit 32 different banks).  The stages run in passes
-// of up to five: in pass p every thread takes groups of 2^b elements 32^p
-// apart and does their b stages in registers (the stages of the row in
-// increasing h), with a CTA barrier between passes.  The row is read once and
-// written once.
+// A CTA holds whole rows; the stages run in passes of up to five: in pass p
+// every thread takes groups of 2^b elements 32^p apart and does their b stages
+// in registers (the stages of the row in increasing h), with a CTA barrier
+// between passes.  The first pass reads its 32-element runs straight from
+// global memory and the last pass writes straight back; the passes between
+// them keep the rows in shared memory as fp32 (element i at word i + i/32, so
+// both the contiguous runs and the strided groups hit 32 different banks).
+// The row is read once and written once.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -56,9 +57,12 @@ template <>
 __device__ __forceinline__ __half from_f32<__half>(float v) { return __float2half_rn(v); }
 
 // One pass: groups of 2^B elements `stride` apart; their B butterfly stages;
-// the final multiply when this is the last pass.
-template <int B>
-__device__ __forceinline__ void pass(float* buf, int pad_n, int nrows, int log2n, int shift, bool last, float c) {
+// the final multiply when this is the last pass.  With `out` set (the last
+// pass of the register path) the results go straight to the rows in global
+// memory: for each t the lanes of a warp hold consecutive columns.
+template <int B, typename T>
+__device__ __forceinline__ void pass(float* buf, int pad_n, int nrows, int log2n, int shift, bool last, float c,
+                                     T* out = nullptr) {
   constexpr int kR = 1 << B;
   const int stride = 1 << shift;
   const int per_row = 1 << (log2n - B);
@@ -85,8 +89,14 @@ __device__ __forceinline__ void pass(float* buf, int pad_n, int nrows, int log2n
 #pragma unroll
       for (int t = 0; t < kR; ++t) v[t] = __fmul_rn(v[t], c);
     }
+    if (out) {
+      T* orow = out + ((size_t)row << log2n);
 #pragma unroll
-    for (int t = 0; t < kR; ++t) rb[padw(base + t * stride)] = v[t];
+      for (int t = 0; t < kR; ++t) orow[base + t * stride] = from_f32<T>(v[t]);
+    } else {
+#pragma unroll
+      for (int t = 0; t < kR; ++t) rb[padw(base + t * stride)] = v[t];
+    }
   }
 }
 
@@ -98,6 +108,72 @@ __global__ void __launch_bounds__(kThreadsH) hadamard_transform_kernel(T* __rest
   const int row0 = blockIdx.x * rows_per_cta;
   const int nrows = min(rows_per_cta, rows - row0);
   T* xr = x + (size_t)row0 * n;
+  const int passes = (log2n + 4) / 5;          // n = 1: none (the multiply by 1 changes nothing)
+  if (log2n >= 5 && (reinterpret_cast<uintptr_t>(x) & 15u) == 0) {
+    // Register path: the first pass takes each 32-element run straight from
+    // global memory (four 16-byte loads per thread; consecutive threads,
+    // consecutive runs), the last pass writes straight back, and only the
+    // passes between them go through shared memory (lane L's 32 words at
+    // 33L .. 33L+31: 32 different banks for each t).
+    for (int g = threadIdx.x; g < nrows << (log2n - 5); g += blockDim.x) {
+      const uint4* src = reinterpret_cast<const uint4*>(xr + ((size_t)g << 5));
+      uint4 w[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) w[q] = src[q];
+      float v[32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t u[4] = {w[q].x, w[q].y, w[q].z, w[q].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[8 * q + 2 * j] = to_f32<T>(u[j] & 0xFFFFu);
+          v[8 * q + 2 * j + 1] = to_f32<T>(u[j] >> 16);
+        }
+      }
+#pragma unroll
+      for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          if ((t & h) == 0) {
+            const float a = v[t], b = v[t + h];
+            v[t] = __fadd_rn(a, b);
+            v[t + h] = __fsub_rn(a, b);
+          }
+        }
+      }
+      if (passes == 1) {
+        uint4* dst = reinterpret_cast<uint4*>(xr + ((size_t)g << 5));
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t o[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            o[j] = bits16(from_f32<T>(__fmul_rn(v[8 * q + 2 * j], c))) |
+                   (bits16(from_f32<T>(__fmul_rn(v[8 * q + 2 * j + 1], c))) << 16);
+          dst[q] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      } else {
+        float* d = buf + (g >> (log2n - 5)) * pad_n + padw((g << 5) & (n - 1));
+#pragma unroll
+        for (int t = 0; t < 32; ++t) d[t] = v[t];
+      }
+    }
+    for (int p = 1; p < passes; ++p) {
+      __syncthreads();
+      const int b = min(5, log2n - 5 * p);
+      const bool last = p == passes - 1;
+      T* out = last ? xr : nullptr;
+      switch (b) {
+        case 1: pass<1>(buf, pad_n, nrows, log2n, 5 * p, last, c, out); break;
+        case 2: pass<2>(buf, pad_n, nrows, log2n, 5 * p, last, c, out); break;
+        case 3: pass<3>(buf, pad_n, nrows, log2n, 5 * p, last, c, out); break;
+        case 4: pass<4>(buf, pad_n, nrows, log2n, 5 * p, last, c, out); break;
+        default: pass<5>(buf, pad_n, nrows, log2n, 5 * p, last, c, out); break;
+      }
+    }
+    return;
+  }
+  // Shared-memory path (n < 32 or a base address without 16-byte alignment).
   // 16-byte accesses (8 elements, inside one row since 8 | n) when the rows
   // allow it; lane L's eight words then sit in banks distinct from the other
   // lanes' (8L + L/4 covers 0..31 once).
@@ -121,16 +197,15 @@ __global__ void __launch_bounds__(kThreadsH) hadamard_transform_kernel(T* __rest
       buf[(e >> log2n) * pad_n + padw(e & (n - 1))] = load_f32(xr + e);
   }
   __syncthreads();
-  const int passes = (log2n + 4) / 5;          // n = 1: none (the multiply by 1 changes nothing)
   for (int p = 0; p < passes; ++p) {
     const int b = min(5, log2n - 5 * p);
     const bool last = p == passes - 1;
     switch (b) {
-      case 1: pass<1>(buf, pad_n, nrows, log2n, 5 * p, last, c); break;
-      case 2: pass<2>(buf, pad_n, nrows, log2n, 5 * p, last, c); break;
-      case 3: pass<3>(buf, pad_n, nrows, log2n, 5 * p, last, c); break;
-      case 4: pass<4>(buf, pad_n, nrows, log2n, 5 * p, last, c); break;
-      default: pass<5>(buf, pad_n, nrows, log2n, 5 * p, last, c); break;
+      case 1: pass<1, T>(buf, pad_n, nrows, log2n, 5 * p, last, c); break;
+      case 2: pass<2, T>(buf, pad_n, nrows, log2n, 5 * p, last, c); break;
+      case 3: pass<3, T>(buf, pad_n, nrows, log2n, 5 * p, last, c); break;
+      case 4: pass<4, T>(buf, pad_n, nrows, log2n, 5 * p, last, c); break;
+      default: pass<5, T>(buf, pad_n, nrows, log2n, 5 * p, last, c); break;
     }
     __syncthreads();
   }
