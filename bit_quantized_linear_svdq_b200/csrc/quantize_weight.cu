@@ -11,9 +11,9 @@
 //   w_hat = fp32(w)                    (exact from bf16), optionally
 //   w_hat = fp32(butterfly_128(w_hat) * fp32(1/sqrt(128)))
 //   scale = e4m3_rne_satfinite(fp32(amax16 / 6)),  code = e2m1_rne_satfinite(fp32(w_hat / scale))
-// with IEEE fp32 divisions (a block whose scale rounds to zero gets codes 0;
-// a block holding NaN gets the NaN scale byte and codes 0, as the activation
-// quantizer's non-finite path).
+// with correctly rounded fp32 divisions (nvfp4_block.cuh: a block whose scale
+// rounds to zero gets codes 0; a block holding a NaN or an infinity takes the
+// IEEE-division path).
 //
 // One CTA of 128 threads covers 32 rows x 128 K elements: four threads per
 // row, 32 consecutive elements (two scale blocks) each, so a warp reads and
@@ -23,6 +23,7 @@
 
 #include "hadamard.cuh"
 #include "kcommon.cuh"
+#include "nvfp4_block.cuh"
 #include "svdq_kernels.h"
 
 namespace svdq {
@@ -30,37 +31,19 @@ namespace {
 
 constexpr int kRowsW = 32, kChunkW = 128, kThreadsW = 128;
 
-// One 16-element block held as 8 packed pairs: scale byte and 16 codes.
-__device__ __forceinline__ uint32_t quant_block_ieee(const uint64_t (&v)[8], uint32_t& w0, uint32_t& w1) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    float r;
-    asm("max.NaN.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(amax), "f"(lo2(v[i])), "f"(hi2(v[i])));
-    amax = r;
-  }
-  const uint32_t sb = cvt_e4m3(__fdiv_rn(amax, 6.0f));
-  const float s = e4m3_to_f32(sb);
-  w0 = w1 = 0u;
-  if (s > 0.0f) {
-    float q[16];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      q[2 * i] = __fdiv_rn(lo2(v[i]), s);
-      q[2 * i + 1] = __fdiv_rn(hi2(v[i]), s);
-    }
-    w0 = cvt_e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
-    w1 = cvt_e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
-  }
-  return sb;
-}
-
 template <bool ROT>
 __global__ void __launch_bounds__(kThreadsW)
     quantize_weight_kernel(const __nv_bfloat16* __restrict__ w, int N, int K, uint8_t* __restrict__ qweight,
                            uint8_t* __restrict__ wscales) {
   __shared__ uint8_t sc[kChunkW / 16][kRowsW];      // [block in chunk][row]
+  __shared__ float2 srec[128];                       // e4m3 code -> {-s, RN(1/s)}
   const int tid = threadIdx.x, rl = tid >> 2, qq = tid & 3;
+  {
+    const float s = e4m3_to_f32((uint32_t)tid);
+    srec[tid] = make_float2(-s, tid ? __frcp_rn(s) : 0.0f);
+  }
+  const float y6 = __frcp_rn(6.0f);
+  __syncthreads();
   const int n0 = blockIdx.y * kRowsW, n = n0 + rl;
   const int k0 = blockIdx.x * kChunkW + 32 * qq;     // first element of this thread's quarter
   uint64_t v[16];
@@ -85,7 +68,7 @@ __global__ void __launch_bounds__(kThreadsW)
     uint64_t blk[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) blk[i] = v[8 * b + i];
-    sbytes |= quant_block_ieee(blk, cw[2 * b], cw[2 * b + 1]) << (8 * b);
+    sbytes |= quantize_any(blk, srec, y6, cw[2 * b], cw[2 * b + 1]) << (8 * b);
   }
   if (n < N) {
     uint2* dst = reinterpret_cast<uint2*>(qweight + (size_t)n * (K / 2) + k0 / 2);   // 8-byte aligned
