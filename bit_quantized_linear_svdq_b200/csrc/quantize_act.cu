@@ -14,19 +14,18 @@
 // Work decomposition.  A CTA owns 128 token rows and a contiguous slice of
 // K; the K slices of one row tile form a thread-block cluster that reduces
 // its partial L in distributed shared memory (fixed order, deterministic).
-// Inside a CTA (one CTA per SM):
-//   producer warp   lane 0, TMA producer: x chunk (128 rows x 128 K, two 128B-swizzled
+// Inside a CTA (320 threads, one CTA per SM):
+//   warp 8 lane 0   TMA producer: x chunk (128 rows x 128 K, two 128B-swizzled
 //                   boxes), proj_down^T chunk (R x 128) and the smooth factors
-//                   into a ring of up to 4 stages; this warp also owns the TMEM
+//                   into a ring of up to 4 stages; warp 8 also owns the TMEM
 //                   allocation.
-//   compute warps   without rotation (16 warps): each thread one 16-channel
-//                   block of two rows; with rotation (8 warps): four threads
-//                   per row (32 K elements each, two rows per chunk in turn):
-//                   smooth (+ rotate),
+//   warps 0-7       without rotation: each thread one 16-channel block of four
+//                   rows; with rotation: four threads per row (32 K elements
+//                   each, two rows per chunk in turn): smooth (+ rotate),
 //                   quantize, write codes/scales to global, and write bf16(x_hat)
 //                   back in place over x in shared memory -- exactly the
 //                   128B-swizzled K-major layout the tensor core reads as A.
-//   MMA warp        lane 0 issues tcgen05.mma (M=128, N=R, K=16, bf16 -> fp32 TMEM)
+//   warp 9 lane 0   issues tcgen05.mma (M=128, N=R, K=16, bf16 -> fp32 TMEM)
 //                   for L on each finished chunk, releasing the stage when done.
 //
 // Exact fp32 division without the divide unit: with y = RN(1/b),
@@ -64,20 +63,18 @@ constexpr int kLamStageBytes = kChunk * 8;         // float4 {-s0,-s1,1/s0,1/s1}
 // chunk's two adjacent scale atoms).
 constexpr int kCodeStageBytes = kRows * kChunk / 2;   // 8 KB
 constexpr int kSfStageBytes = 2 * kSfAtomBytes;       // 1 KB
-// Thread layout: the compute warps, then the TMA producer warp and the MMA
-// warp.  The unrotated path has 16 compute warps, each thread two rows of one
-// 16-channel block column, the smoothing operands read from shared memory per
-// channel pair rather than held (96 registers; the kernel time is unchanged
-// against 8 warps of four rows, and the step with the GEMM that follows is
-// 0.8 us shorter).  The rotated path has 8 compute warps with four threads to
-// each row, two rows per chunk in turn: with ten warps a thread gets at most
-// 168 registers (each SM sub-partition holds three of the warps), and a
-// 64-value slice of the rotation block per thread spilled.
+// Thread layout: 8 compute warps, then the TMA producer warp and the MMA
+// warp.  The unrotated path gives each thread four rows of one 16-channel
+// block column (measured faster than 16 warps of two rows, which need fewer
+// registers than the four-row chains want); the rotated path gives four
+// threads to each row, two rows per chunk in turn: with ten warps a thread
+// gets at most 168 registers (each SM sub-partition holds three of the warps),
+// and a 64-value slice of the rotation block per thread spilled.
 template <bool ROT>
 struct QCfg {
-  static constexpr int kComputeWarps = ROT ? 8 : 16;
+  static constexpr int kComputeWarps = 8;
   static constexpr int kComputeThreads = 32 * kComputeWarps;
-  static constexpr int kRowsPerThread = 2;     // unrotated: rows r0 + (128 / 4) * rr; rotated: row4, row4 + 64
+  static constexpr int kRowsPerThread = ROT ? 2 : 4;     // unrotated: rows r0 + (128 / 4) * rr; rotated: row4, row4 + 64
   static constexpr int kProducerWarp = kComputeWarps, kMmaWarp = kComputeWarps + 1;
   static constexpr int kThreads = 32 * (kComputeWarps + 2);
 };
@@ -189,6 +186,13 @@ __device__ __forceinline__ void smooth_cols(uint8_t* xs, const float4* lam4, con
                                             uint32_t (&cw)[kColRowsPerThread][2], uint32_t (&sb)[kColRowsPerThread]) {
   constexpr int RPT = kColRowsPerThread;
   const int j = t & 7, r0 = t >> 3;
+  uint64_t nb[8], yb[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 l = lam4[8 * i + j];                 // pair 8j + i (see lam_slot)
+    nb[i] = pk2(l.x, l.y);
+    yb[i] = pk2(l.z, l.w);
+  }
   // The thread's rows are all loaded before any is written back, and the
   // common path has no per-row branch, so the rows' dependency chains
   // (divide, amax, scale, divide, convert) overlap.
@@ -205,15 +209,10 @@ __device__ __forceinline__ void smooth_cols(uint8_t* xs, const float4* lam4, con
   float amax[RPT];
   bool finite = true;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float4 l = lam4[8 * i + j];                 // pair 8j + i (see lam_slot)
-    const uint64_t nbi = pk2(l.x, l.y), ybi = pk2(l.z, l.w);
-#pragma unroll
-    for (int rr = 0; rr < RPT; ++rr)
-      v[rr][i] = NEG ? div_mk2(bf16x2_to_f2(xin[rr][i]), nbi, ybi) : div_rn2(bf16x2_to_f2(xin[rr][i]), nbi, ybi);
-  }
-#pragma unroll
   for (int rr = 0; rr < RPT; ++rr) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      v[rr][i] = NEG ? div_mk2(bf16x2_to_f2(xin[rr][i]), nb[i], yb[i]) : div_rn2(bf16x2_to_f2(xin[rr][i]), nb[i], yb[i]);
     amax[rr] = amax8(v[rr]);
     finite = finite && (amax[rr] < 3.0e38f);
   }
@@ -231,8 +230,7 @@ __device__ __forceinline__ void smooth_cols(uint8_t* xs, const float4* lam4, con
       } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float4 l = lam4[8 * i + j];
-          const float s0 = NEG ? l.x : -l.x, s1 = NEG ? l.y : -l.y;
+          const float s0 = NEG ? lo2(nb[i]) : -lo2(nb[i]), s1 = NEG ? hi2(nb[i]) : -hi2(nb[i]);
           v[rr][i] = pk2(__fdiv_rn(__uint_as_float(xin[rr][i] << 16), s0),
                          __fdiv_rn(__uint_as_float(xin[rr][i] & 0xFFFF0000u), s1));
         }
