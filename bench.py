@@ -22,6 +22,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -63,16 +64,37 @@ def gemm_bytes(M, K, N, R):
     return M * K / 2 + M * K / 16 + 2.0 * M * R + N * K / 2 + N * K / 16 + 2.0 * N * R + 4.0 * N + 2.0 * M * N
 
 
+def source_digest(path):
+    """sha256 over a kernel source and every local header it includes,
+    transitively, in first-seen order."""
+    seen, order = set(), []
+
+    def walk(p):
+        if p in seen or not os.path.exists(p):
+            return
+        seen.add(p)
+        order.append(p)
+        with open(p, "r", errors="replace") as f:
+            for inc in re.findall(r'^\s*#\s*include\s+"([^"]+)"', f.read(), re.M):
+                walk(os.path.join(os.path.dirname(p), inc))
+
+    walk(os.path.join(ROOT, path))
+    h = hashlib.sha256()
+    for p in order:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def measured_traffic(workload, kernel):
     """DRAM bytes (read + write) per launch from the ncu capture recorded in
     profiles/traffic.json, or None when there is none or the kernel's source
-    has changed since it was taken."""
+    (its .cu file and the local headers it includes) has changed since."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f)[workload][kernel]
-        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
-                return None
+        if source_digest(rec["source"]) != rec["source_sha256"]:
+            return None
         return rec["dram_bytes_per_launch"]
     except (OSError, KeyError, ValueError):
         return None
@@ -404,19 +426,23 @@ def run_ours(args, world, rank, local):
     g_tf = g_flops / (us_g * 1e-6) / 1e12
     kernels = {
         "quantize_act": {"us": us_q, "bound": "hbm", "algorithmic_bytes": quant_bytes(M, K, R),
-                         "achieved_gbs": q_gbs, "frac_of_hbm": q_gbs / pk["hbm_gbs"]},
+                         "achieved_gbs": q_gbs, "frac_of_hbm": q_gbs / pk["hbm_gbs"],
+                         "traffic": measured_traffic(ck.name, "quantize_act")},
         "quantize_weight": {"us": us_wq, "bound": "hbm", "algorithmic_bytes": wq_bytes,
                             "achieved_gbs": wq_bytes / (us_wq * 1e-6) / 1e9,
                             "frac_of_hbm": wq_bytes / (us_wq * 1e-6) / 1e9 / pk["hbm_gbs"],
+                            "traffic": measured_traffic(ck.name, "quantize_weight"),
                             "note": "offline step (dense weight -> NVFP4), on this layer's weight shape"},
         "hadamard_transform": {"us": us_ht, "bound": "hbm", "algorithmic_bytes": ht_bytes,
                                "achieved_gbs": ht_bytes / (us_ht * 1e-6) / 1e9,
                                "frac_of_hbm": ht_bytes / (us_ht * 1e-6) / 1e9 / pk["hbm_gbs"],
+                               "traffic": measured_traffic(ck.name, "hadamard_transform"),
                                "note": f"standalone transform, in place on {M} x {HN} bf16"},
         "gemm_nvfp4": {"us": us_g, "bound": "tensor", "variant": gemm_variant(ck), "algorithmic_flops": g_flops,
                        "achieved_tflops": g_tf, "frac_of_fp4": g_tf / fp4_peak,
                        "algorithmic_bytes": gemm_bytes(M, K, N, R),
-                       "achieved_gbs": gemm_bytes(M, K, N, R) / (us_g * 1e-6) / 1e9},
+                       "achieved_gbs": gemm_bytes(M, K, N, R) / (us_g * 1e-6) / 1e9,
+                       "traffic": measured_traffic(ck.name, "gemm_nvfp4")},
     }
     if us_g >= us_q:
         roof = {"kernel": "gemm_nvfp4 (" + gemm_variant(ck) + ")", "bound": "tensor", "achieved": g_tf, "peak": fp4_peak,
