@@ -22,7 +22,7 @@ __all__ = [
     "SvdqError", "svdq_linear_desc", "load_library", "library_path", "exported_names",
     "svdq_linear_create", "svdq_linear_destroy", "svdq_workspace_bytes", "svdq_quantize_act",
     "svdq_linear_forward", "svdq_linear_forward_host", "svdq_linear_forward_quantize",
-    "svdq_linear_forward_gemm", "svdq_device_status", "svdq_status_string",
+    "svdq_linear_forward_gemm", "svdq_linear_gemm_kernel", "svdq_device_status", "svdq_status_string",
     "svdq_last_error", "svdq_version", "svdq_quantize_weight", "quantize_weight", "svdq_hadamard_transform", "hadamard_transform", "SVDQLinear", "STATUS",
 ]
 
@@ -85,6 +85,7 @@ def load_library() -> ctypes.CDLL:
         "svdq_linear_forward_host": (ci, [vp, vp, ci, vp, vp, vp, vp, vp]),
         "svdq_linear_forward_quantize": (ci, [vp, vp, ci, vp, vp]),
         "svdq_linear_forward_gemm": (ci, [vp, ci, vp, vp, vp]),
+        "svdq_linear_gemm_kernel": (ctypes.c_char_p, [vp, ci]),
         "svdq_linear_forward_noalloc": (ci, [vp, vp, ci, vp, vp]),
         "svdq_device_status": (ci, [vp, ctypes.POINTER(ci)]),
         "svdq_status_string": (ctypes.c_char_p, [ci]),
@@ -168,6 +169,11 @@ def svdq_linear_forward_quantize(handle, x_ptr, M, workspace_ptr, stream=None) -
 def svdq_linear_forward_gemm(handle, M, y_ptr, workspace_ptr, stream=None) -> None:
     _check(load_library().svdq_linear_forward_gemm(handle, M, y_ptr, workspace_ptr, _stream(stream)),
            "svdq_linear_forward_gemm")
+
+
+def svdq_linear_gemm_kernel(handle, M) -> str:
+    """Name of the kernel svdq_linear_forward_gemm launches for M rows."""
+    return (load_library().svdq_linear_gemm_kernel(handle, M) or b"").decode()
 
 
 def svdq_linear_forward_host(handle, x_host_ptr, M, y_host_ptr, x_dev_ptr, y_dev_ptr, workspace_ptr,
@@ -311,6 +317,10 @@ class SVDQLinear:
 
     def device_status(self) -> int:
         return svdq_device_status(self.handle)
+
+    def gemm_kernel(self, M: int) -> str:
+        """Name of the kernel the GEMM stage launches for M rows."""
+        return svdq_linear_gemm_kernel(self.handle, M)
 
     def close(self) -> None:
         if getattr(self, "handle", None):

@@ -106,6 +106,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  // The weights (library-owned, written once at create time, which
+  // synchronizes) do not depend on the previous kernel: the first tile's
+  // first stages of weight codes and scale atoms start streaming now, while
+  // that kernel (the activation quantizer) may still be running.  The stage
+  // barriers are armed with the whole stage; the token half follows in the
+  // producer loop.
+  const int npre = (int)blockIdx.x < p.n_tiles ? min(kStages, p.k_tiles) : 0;
+  if (tid == 0 && npre > 0) {
+    const int n0 = (int)blockIdx.x * BM;
+    prefetch_tmap(&tm_w);
+    for (int i = 0; i < npre; ++i) {
+      uint8_t* st = ring + i * kStageBytes;
+      const uint32_t fb = smem_u32(&full[i]);
+      mbar_arrive_expect_tx(fb, kStageBytes);
+      tma_load_2d(smem_u32(st), &tm_w, fb, i * kKTileBytes, n0);
+      bulk_load(smem_u32(st + kWBytes + kXBytes),
+                p.sfb + ((size_t)blockIdx.x * p.ka_pad + (size_t)i * kAtoms) * kSfAtomBytes, kSfwBytes, fb);
+    }
+  }
   // Everything above overlaps the previous kernel's tail (programmatic
   // dependent launch); nothing below runs before it has completed.
   griddep_wait();
@@ -122,7 +141,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   int issued = 0, lr_issued = 0;
   if (warp == kProdWarp) {
     if (lane == 0) {
-      prefetch_tmap(&tm_w);
       prefetch_tmap(&tm_x);
       prefetch_tmap(&tm_pu);
       prefetch_tmap(&tm_l);
@@ -138,11 +156,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t* st = ring + s * kStageBytes;
           const uint32_t fb = smem_u32(&full[s]);
-          mbar_arrive_expect_tx(fb, kStageBytes);
-          tma_load_2d(smem_u32(st), &tm_w, fb, kt * kKTileBytes, n0);
+          if (g >= npre) {                         // else armed, weight half in flight since the prologue
+            mbar_arrive_expect_tx(fb, kStageBytes);
+            tma_load_2d(smem_u32(st), &tm_w, fb, kt * kKTileBytes, n0);
+            bulk_load(smem_u32(st + kWBytes + kXBytes),
+                      p.sfb + ((size_t)tile * p.ka_pad + (size_t)kt * kAtoms) * kSfAtomBytes, kSfwBytes, fb);
+          }
           tma_load_2d(smem_u32(st + kWBytes), &tm_x, fb, kt * kKTileBytes, 0);
-          bulk_load(smem_u32(st + kWBytes + kXBytes),
-                    p.sfb + ((size_t)tile * p.ka_pad + (size_t)kt * kAtoms) * kSfAtomBytes, kSfwBytes, fb);
           bulk_load(smem_u32(st + kWBytes + kXBytes + kSfwBytes), p.sfa + (size_t)kt * kAtoms * kSfAtomBytes,
                     kSfxBytes, fb);
           issued = g + 1;

@@ -110,6 +110,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(mma_done), 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // The weights (library-owned, written once at create time, which
+    // synchronizes) do not depend on the previous kernel: the first stages'
+    // weight codes and scale atoms start streaming now, while that kernel
+    // (the activation quantizer) may still be running.  Each stage's barrier
+    // is armed with the whole stage; its activation half follows below.
+    prefetch_tmap(&tm_b);
+    for (int i = 0; i < min(nk, kStages); ++i) {
+      uint8_t* st = stages + i * kStageBytes;
+      const uint32_t fb = smem_u32(&full[i]);
+      const int kt = kt0 + i;
+      mbar_arrive_expect_tx(fb, kStageBytes);
+      tma_load_2d(smem_u32(st + kABytes), &tm_b, fb, kt * kKTileBytes, n0);
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        bulk_load(smem_u32(st + kABytes + kBBytes + kSfaBytes + h * (kSfbBytes / 2)),
+                  p.sfb + ((size_t)(2 * nt + h) * p.ka_pad + (size_t)kt * kAtoms) * kSfAtomBytes, kSfbBytes / 2, fb);
+    }
   }
   // Everything above overlaps the previous kernel's tail (programmatic
   // dependent launch); nothing below runs before it has completed.
@@ -128,21 +145,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       prefetch_tmap(&tm_a);
-      prefetch_tmap(&tm_b);
       for (int i = 0; i < nk; ++i) {
         const int s = i % kStages, n = i / kStages, kt = kt0 + i;
         if (n >= 1 && !wait_bounded(smem_u32(&empty[s]), (n - 1) & 1, abort_flag, p.err, kErrGemmTimeout)) break;
         uint8_t* st = stages + s * kStageBytes;
         const uint32_t fb = smem_u32(&full[s]);
-        mbar_arrive_expect_tx(fb, kStageBytes);
+        if (n >= 1) {                              // the first kStages stages: armed, weights in flight
+          mbar_arrive_expect_tx(fb, kStageBytes);
+          tma_load_2d(smem_u32(st + kABytes), &tm_b, fb, kt * kKTileBytes, n0);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            bulk_load(smem_u32(st + kABytes + kBBytes + kSfaBytes + h * (kSfbBytes / 2)),
+                      p.sfb + ((size_t)(2 * nt + h) * p.ka_pad + (size_t)kt * kAtoms) * kSfAtomBytes, kSfbBytes / 2,
+                      fb);
+        }
         tma_load_2d(smem_u32(st), &tm_a, fb, kt * kKTileBytes, m0);
-        tma_load_2d(smem_u32(st + kABytes), &tm_b, fb, kt * kKTileBytes, n0);
         bulk_load(smem_u32(st + kABytes + kBBytes),
                   p.sfa + ((size_t)mt * p.ka_pad + (size_t)kt * kAtoms) * kSfAtomBytes, kSfaBytes, fb);
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          bulk_load(smem_u32(st + kABytes + kBBytes + kSfaBytes + h * (kSfbBytes / 2)),
-                    p.sfb + ((size_t)(2 * nt + h) * p.ka_pad + (size_t)kt * kAtoms) * kSfAtomBytes, kSfbBytes / 2, fb);
         issued = i + 1;
       }
     }

@@ -19,6 +19,7 @@ struct svdq_linear {
   int K, N, R, Kp, ka_pad, k_tiles, rotate_block;
   uint8_t* qw;            // (N, Kp/2) packed E2M1, rows zero-padded to Kp
   uint8_t* sfb;           // weight scale tiles: ceil(N/128) x ka_pad replicated atoms of 2 KB
+  uint8_t* sfr;           // (N, Kp/16) the same scales row-major, zero beyond K/16 (few-row CUDA-core product)
   __nv_bfloat16* pdT;     // proj_down^T (R, Kp), zero-padded
   __nv_bfloat16* pu;      // proj_up (N, R)
   float4* lam4;           // (Kp/2) {-s_k, -s_k+1, 1/s_k, 1/s_k+1} per channel pair, padded with s = 1
@@ -31,6 +32,7 @@ struct svdq_linear {
   bool splitk;            // few rows: split-K GEMM over a cluster (unless SVDQ_SPLITK=0 at create)
   bool pair;              // more than 128 rows: 256 x 256 tiles on CTA pairs (unless SVDQ_GEMM_PAIR=0 at create)
   bool narrow;            // 9..32 rows: y^T on 128-column full-K tiles (unless SVDQ_GEMM_NARROW=0 at create)
+  bool gemv;              // 1..4 rows: CUDA-core matrix-vector product (unless SVDQ_GEMV=0 at create)
   int lr_row_bytes;       // 128 x 256 GEMM: bytes per row of its L / proj_up' tiles
   int pair_row_bytes;     // pair GEMM: bytes per row of one L / proj_up' box
   unsigned* err;          // device error word
@@ -106,11 +108,13 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 // ---------------------------------------------------------------- create-time repack kernels
 
-// Weight scales into replicated tensor-core atoms.  Columns whose alpha is 0
-// get zero scales: their main product is multiplied by 0 anyway, and a zero
-// there lets the 128 x 256 GEMM give them alpha' = 1 with y = L proj_up^T.
+// Weight scales into replicated tensor-core atoms, and row-major (N, Kp/16)
+// for the few-row CUDA-core product.  Columns whose alpha is 0 get zero
+// scales: their main product is multiplied by 0 anyway, and a zero there lets
+// the 128 x 256 GEMM give them alpha' = 1 with y = L proj_up^T.
 __global__ void repack_weight_scales(const uint8_t* __restrict__ wscales, const float* __restrict__ alpha,
-                                     uint8_t* __restrict__ sfb, int K16, int N, int ka_pad, unsigned* bad) {
+                                     uint8_t* __restrict__ sfb, uint8_t* __restrict__ sfr, int K16, int N,
+                                     int ka_pad, int sfr_pitch, unsigned* bad) {
   const long long total = (long long)K16 * N;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
     const int kb = (int)(i / N), n = (int)(i % N);
@@ -118,6 +122,7 @@ __global__ void repack_weight_scales(const uint8_t* __restrict__ wscales, const 
     if ((w & 0x7F) == 0x7F) atomicOr(bad, 1u);       // e4m3 NaN
     const uint8_t b = alpha[n] == 0.0f ? 0 : w;
     sfb[((size_t)(n >> 7) * ka_pad + (kb >> 2)) * svdq::kSfAtomBytes + svdq::sf_atom_offset(n & 127, kb & 3)] = b;
+    sfr[(size_t)n * sfr_pitch + kb] = b;
   }
 }
 
@@ -214,6 +219,7 @@ void free_handle(svdq_linear* h) {
   if (!h) return;
   cudaFree(h->qw);
   cudaFree(h->sfb);
+  cudaFree(h->sfr);
   cudaFree(h->pdT);
   cudaFree(h->pu);
   cudaFree(h->lam4);
@@ -320,6 +326,7 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
 
   CREATE_CUDA(cudaMalloc(&h->qw, (size_t)d->N * (h->Kp / 2)));
   CREATE_CUDA(cudaMalloc(&h->sfb, (size_t)n_tiles_even * h->ka_pad * svdq::kSfAtomBytes));
+  CREATE_CUDA(cudaMalloc(&h->sfr, (size_t)d->N * (h->Kp / 16)));
   CREATE_CUDA(cudaMalloc(&h->pdT, (size_t)d->R * h->Kp * 2));
   CREATE_CUDA(cudaMalloc(&h->pu, (size_t)d->N * d->R * 2));
   CREATE_CUDA(cudaMalloc(&h->lam4, (size_t)(h->Kp / 2) * sizeof(float4)));
@@ -342,12 +349,14 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
   CREATE_CUDA(cudaMemcpy2DAsync(h->qw, h->Kp / 2, d->qweight, d->K / 2, d->K / 2, d->N, cudaMemcpyDeviceToDevice,
                                 stream));
   CREATE_CUDA(cudaMemsetAsync(h->sfb, 0, (size_t)n_tiles_even * h->ka_pad * svdq::kSfAtomBytes, stream));
+  CREATE_CUDA(cudaMemsetAsync(h->sfr, 0, (size_t)d->N * (h->Kp / 16), stream));
   prepare_alpha<<<grid_for(Npad), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(d->wcscales),
                                                      static_cast<const __nv_bfloat16*>(d->wtscale), h->alpha, d->N,
                                                      Npad);
   CREATE_CUDA(cudaGetLastError());
   repack_weight_scales<<<grid_for((long long)(d->K / 16) * d->N), 256, 0, stream>>>(
-      static_cast<const uint8_t*>(d->wscales), h->alpha, h->sfb, d->K / 16, d->N, h->ka_pad, h->err + 1);
+      static_cast<const uint8_t*>(d->wscales), h->alpha, h->sfb, h->sfr, d->K / 16, d->N, h->ka_pad, h->Kp / 16,
+      h->err + 1);
   CREATE_CUDA(cudaGetLastError());
   transpose_proj_down<<<grid_for((long long)d->R * h->Kp), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(d->proj_down), h->pdT, d->K, d->R, h->Kp);
@@ -381,6 +390,8 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
     h->pair = foldable && !(pr && pr[0] == '0');
     const char* nw = std::getenv("SVDQ_GEMM_NARROW");
     h->narrow = h->n256 && !(nw && nw[0] == '0');
+    const char* gv = std::getenv("SVDQ_GEMV");
+    h->gemv = !(gv && gv[0] == '0');
     h->pair_row_bytes = svdq::gemm_pair_lr_row_bytes(d->R);
     h->lr_row_bytes = svdq::gemm_n256_lr_row_bytes(d->R);
   }
@@ -518,9 +529,48 @@ int num_sms() {
   return n;
 }
 
+// Which GEMM kernel serves M rows on this handle (S: split-K cluster size).
+enum class GemmKind { gemv, narrow, splitk, pair, n256, lr };
+
+GemmKind pick_gemm(const svdq_linear* h, int M, int* S) {
+  *S = 1;
+  // 1..4 rows: the weight read bounds the product; CUDA cores, no tiles.
+  if (h->gemv && svdq::gemv_applies(M, h->Kp, h->R)) return GemmKind::gemv;
+  // 9..32 rows (R <= 32): y^T on 128-column tiles over the whole of K.
+  if (h->narrow && svdq::gemm_narrow_applies(M, h->R)) return GemmKind::narrow;
+  // Few rows: split K over a cluster so the weight read is spread over the GPU.
+  if (h->splitk) *S = svdq::gemm_splitk_slices(M, h->N, h->R, h->k_tiles, num_sms());
+  if (*S > 1) return GemmKind::splitk;
+  if (h->pair && M > 128 && svdq::gemm_pair_available(h->R)) return GemmKind::pair;
+  if (h->n256) return GemmKind::n256;
+  return GemmKind::lr;
+}
+
 svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, cudaStream_t stream) {
   const WsLayout w = ws_layout(h, M);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int S = 1;
+  const GemmKind kind = pick_gemm(h, M, &S);
+  if (kind == GemmKind::gemv) {
+    svdq::GemvLaunch v;
+    v.qw = h->qw;
+    v.sfr = h->sfr;
+    v.codes = ws + w.codes;
+    v.sfa = ws + w.sfa;
+    v.lowrank = ws + w.lr;
+    v.pu = h->pu;
+    v.alpha = h->alpha;
+    v.y = y;
+    v.M = M;
+    v.N = h->N;
+    v.K = h->K;
+    v.Kp = h->Kp;
+    v.R = h->R;
+    v.num_sms = num_sms();
+    cudaError_t e = svdq::launch_gemv_nvfp4(v, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "gemv launch");
+    return SVDQ_OK;
+  }
   svdq::GemmLaunch g;
   std::memset(&g, 0, sizeof(g));
   svdq_status s;
@@ -536,8 +586,7 @@ svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, 
   g.R = h->R;
   g.k_tiles = h->k_tiles;
   g.ka_pad = h->ka_pad;
-  // 9..32 rows (R <= 32): y^T on 128-column tiles over the whole of K.
-  if (h->narrow && svdq::gemm_narrow_applies(M, h->R)) {
+  if (kind == GemmKind::narrow) {
     if ((s = make_tmap(&g.tm_a, ws + w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->Kp / 2, M, h->Kp / 2, 128, 32)) !=
         SVDQ_OK)
       return s;
@@ -551,16 +600,14 @@ svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, 
     if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
     return SVDQ_OK;
   }
-  // Few rows: split K over a cluster so the weight read is spread over the GPU.
-  const int S = h->splitk ? svdq::gemm_splitk_slices(M, h->N, h->R, h->k_tiles, num_sms()) : 1;
-  if (S > 1) {
+  if (kind == GemmKind::splitk) {
     g.tm_b = h->tm_b256;
     g.alpha = h->alpha;
     cudaError_t e = svdq::launch_gemm_nvfp4_splitk(g, ws + w.lr, h->pu, S, stream);
     if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
     return SVDQ_OK;
   }
-  if (h->pair && M > 128 && svdq::gemm_pair_available(h->R)) {
+  if (kind == GemmKind::pair) {
     g.tm_b = h->tm_b;
     if ((s = make_tmap(&g.tm_l, ws + w.lr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->R, M, (uint64_t)h->R * 2,
                        h->pair_row_bytes / 2, 128, lr_swizzle(h->pair_row_bytes))) != SVDQ_OK)
@@ -574,7 +621,7 @@ svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, 
     if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
     return SVDQ_OK;
   }
-  if (h->n256) {
+  if (kind == GemmKind::n256) {
     g.tm_b = h->tm_b256;
     if ((s = make_tmap(&g.tm_l, ws + w.lr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->R, M, (uint64_t)h->R * 2,
                        h->lr_row_bytes / 2, 128, lr_swizzle(h->lr_row_bytes))) != SVDQ_OK)
@@ -627,6 +674,24 @@ svdq_status svdq_linear_forward_quantize(const svdq_linear* h, const void* x, in
   if (s != SVDQ_OK || M == 0) return s;
   if (!x || !aligned16(x)) return SVDQ_ERR_INVALID_ARG;
   return forward_quantize(h, x, M, workspace, static_cast<cudaStream_t>(stream));
+}
+
+const char* svdq_linear_gemm_kernel(const svdq_linear* h, int M) {
+  if (!h || M <= 0) return "";
+  int S = 1;
+  switch (pick_gemm(h, M, &S)) {
+    case GemmKind::gemv: return "gemv_nvfp4_kernel (CUDA cores, 1-4 rows)";
+    case GemmKind::narrow: return "gemm_nvfp4_narrow_kernel (y^T on 128 x 32 tiles over the whole of K)";
+    case GemmKind::splitk:
+      return S == 8 ? "gemm_nvfp4_splitk_kernel (128 x 256 tiles, K split over 8-CTA clusters)"
+                    : (S == 4 ? "gemm_nvfp4_splitk_kernel (128 x 256 tiles, K split over 4-CTA clusters)"
+                              : "gemm_nvfp4_splitk_kernel (128 x 256 tiles, K split over 2-CTA clusters)");
+    case GemmKind::pair:
+      return "gemm_nvfp4_pair_kernel (256 x 256 tiles on 2-CTA clusters, tcgen05 cta_group::2, alpha folded)";
+    case GemmKind::n256: return "gemm_nvfp4_n256_kernel (128 x 256 tiles, alpha folded)";
+    case GemmKind::lr: return "gemm_nvfp4_lr_kernel (128 x 128 tiles)";
+  }
+  return "";
 }
 
 svdq_status svdq_linear_forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, void* stream) {

@@ -88,6 +88,27 @@ cudaError_t launch_gemm_nvfp4_n256(const GemmLaunch& p, cudaStream_t stream);
 //   tm_l   L: box {lr_row_bytes / 2, 32}, swizzle of lr_row_bytes
 //   tm_pu  proj_up' (N, R): box {lr_row_bytes / 2, 128}, same swizzle
 bool gemm_narrow_applies(int M, int R);
+
+// 1..kGemvMaxRows token rows on CUDA cores (the product is a matrix-vector
+// product bound by the weight read): weight codes (N, Kp/2), a row-major copy
+// of the weight block scales (N, Kp/16), the activation codes and scale atoms
+// the quantizer wrote, L (M, R), proj_up (N, R), the plain alpha (N).
+constexpr int kGemvMaxRows = 4;
+struct GemvLaunch {
+  const uint8_t* qw;
+  const uint8_t* sfr;
+  const uint8_t* codes;
+  const uint8_t* sfa;
+  const void* lowrank;
+  const void* pu;
+  const float* alpha;
+  void* y;
+  int M, N, K, Kp, R;
+  int num_sms;
+};
+size_t gemv_smem_bytes(int M, int Kp, int R);
+bool gemv_applies(int M, int Kp, int R);
+cudaError_t launch_gemv_nvfp4(const GemvLaunch& L, cudaStream_t stream);
 cudaError_t launch_gemm_nvfp4_narrow(const GemmLaunch& p, cudaStream_t stream);
 
 // The same product on 256 x 256 tiles, each computed by a 2-CTA cluster with

@@ -142,6 +142,15 @@ SVDQ_API svdq_status svdq_linear_forward_gemm(const svdq_linear* h, int M, void*
                                               void* workspace, void* stream);
 
 /*
+ * svdq_linear_gemm_kernel -- static text naming the kernel that
+ * svdq_linear_forward_gemm launches for M rows on this handle ("" for a NULL
+ * handle or M <= 0).  The choice depends on M, N, K, R, the create-time
+ * switches and the device's SM count, and is made by the same function the
+ * launch uses.  Host-only; launches nothing.
+ */
+SVDQ_API const char* svdq_linear_gemm_kernel(const svdq_linear* h, int M);
+
+/*
  * svdq_linear_forward_host -- end-to-end call on HOST buffers: copies x_host
  * (M, K bf16) to x_dev, runs svdq_linear_forward into y_dev, copies y_dev to
  * y_host (M, N bf16) and synchronizes `stream` before returning.  The copies

@@ -21,9 +21,15 @@ def test_exports_every_declared_symbol(lib):
         "svdq_linear_create", "svdq_linear_destroy", "svdq_workspace_bytes", "svdq_quantize_act",
         "svdq_linear_forward", "svdq_linear_forward_host", "svdq_device_status", "svdq_status_string",
         "svdq_last_error", "svdq_version", "svdq_linear_forward_quantize", "svdq_linear_forward_gemm",
-        "svdq_linear_forward_noalloc", "svdq_quantize_weight", "svdq_hadamard_transform"}
+        "svdq_linear_forward_noalloc", "svdq_quantize_weight", "svdq_hadamard_transform",
+        "svdq_linear_gemm_kernel"}
     for n in names:
         assert hasattr(lib, n), n
+
+
+def test_gemm_kernel_query_without_handle(lib):
+    # Host-only query: a NULL handle or M <= 0 names no kernel.
+    assert S.svdq_linear_gemm_kernel(None, 1) == ""
 
 
 def test_status_strings_and_version(lib):

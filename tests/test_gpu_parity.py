@@ -253,14 +253,16 @@ def test_full_workload_parity(name):
 # ------------------------------------------------------------------ ragged shapes and edge cases
 
 def _select_gemm(kernel, monkeypatch):
-    """"auto": the library's choice (alpha folded: 9..32 rows with R <= 32 ->
-    y^T on 128-column full-K tiles; above 128 rows -> 256 x 256 tiles on CTA pairs;
-    otherwise split-K over a cluster for at most 32 rows, 128 x 256 tiles for
-    R <= 32, 128 x 128 tiles); "splitk": the same without the y^T kernel,
-    so split-K serves every few-row shape; "n256" / "n128": the one-CTA
+    """"auto": the library's choice (1..4 rows -> the CUDA-core matrix-vector
+    product; alpha folded: 9..32 rows with R <= 32 -> y^T on 128-column full-K
+    tiles; above 128 rows -> 256 x 256 tiles on CTA pairs; otherwise split-K
+    over a cluster for at most 32 rows, 128 x 256 tiles for R <= 32, 128 x 128
+    tiles); "splitk": the same without the CUDA-core and y^T kernels, so
+    split-K serves every few-row shape; "n256" / "n128": the one-CTA
     persistent kernels alone."""
     if kernel in ("splitk", "n256", "n128"):
         monkeypatch.setenv("SVDQ_GEMM_NARROW", "0")
+        monkeypatch.setenv("SVDQ_GEMV", "0")
     if kernel in ("n256", "n128"):
         monkeypatch.setenv("SVDQ_SPLITK", "0")
         monkeypatch.setenv("SVDQ_GEMM_PAIR", "0")
@@ -284,6 +286,9 @@ def _select_gemm(kernel, monkeypatch):
     (520, 512, 384, 96, 128),   # pair tiles with two rank boxes, three stages, rotation
     (20, 512, 300, 32, 0),      # 9..32 rows: y^T on 128-column tiles, ragged N
     (29, 768, 136, 16, 128),    # the same with rotation, R = 16
+    (2, 4096, 1000, 32, 0),     # 1..4 rows: CUDA-core product, ragged N
+    (4, 9216, 300, 64, 128),    # the same over three 4096-element passes, rotation, R = 64
+    (3, 1040, 77, 16, 0),       # K % 32 == 16 (half-masked last piece), R = 16
 ])
 @pytest.mark.parametrize("kernel", ["auto", "splitk", "n256", "n128"])
 def test_ragged_shapes(M, K, N, R, rot, kernel, monkeypatch):
@@ -297,14 +302,18 @@ def test_ragged_shapes(M, K, N, R, rot, kernel, monkeypatch):
     check_forward(layer, ck)
 
 
+@pytest.mark.parametrize("M", [150, 2])
 @pytest.mark.parametrize("kernel", ["auto", "splitk", "n256", "n128"])
-def test_zero_alpha_columns(kernel, monkeypatch):
+def test_zero_alpha_columns(M, kernel, monkeypatch):
     """Columns with wcscales = 0 reduce to the rank-R branch alone, in every
     GEMM kernel (the folded one gives them alpha' = 1 and zero weight scales)."""
     _select_gemm(kernel, monkeypatch)
-    ck = synthetic.make_checkpoint(150, 512, 520, 32, seed=12, wcscales="uniform",
-                                   name="zero_alpha_150x512x520_r32")
-    zero_cols = np.array([0, 1, 127, 128, 255, 256, 300, 511, 512, 519])
+    ck = synthetic.make_checkpoint(M, 512, 520, 32, seed=12, wcscales="uniform",
+                                   name=f"zero_alpha_{M}x512x520_r32")
+    # Tile edges plus every seventh column: with two rows the check still
+    # averages over ~170 outputs of the rank-R branch, whose bf16 L and y
+    # roundings alone give ~3e-3 (20 outputs gave 5.3e-3 on a correct kernel).
+    zero_cols = np.unique(np.concatenate([[0, 1, 127, 128, 255, 256, 300, 511, 512, 519], np.arange(3, 520, 7)]))
     ck.wcscales = ck.wcscales.copy()
     ck.wcscales[zero_cols] = 0
     layer = make_layer(ck)
@@ -404,3 +413,15 @@ def test_runtime_argument_errors():
     with pytest.raises(S.SvdqError) as e:
         make_layer(bad)
     assert e.value.status == 1
+
+
+def test_gemm_kernel_query():
+    """svdq_linear_gemm_kernel names the kernel the dispatch picks (K = N =
+    3072, R = 32: the attention-projection shape)."""
+    ck = synthetic.make_checkpoint(8, 3072, 3072, 32, seed=21, name="query_8x3072x3072_r32")
+    layer = make_layer(ck)
+    for M, expect in [(1, "gemv_nvfp4"), (4, "gemv_nvfp4"), (5, "splitk"), (20, "narrow"), (100, "n256"),
+                      (300, "pair")]:
+        name = layer.gemm_kernel(M)
+        assert expect in name, (M, name)
+    assert layer.gemm_kernel(0) == ""
