@@ -65,8 +65,10 @@ def gemm_bytes(M, K, N, R):
 
 
 def source_digest(path):
-    """sha256 over a kernel source and every local header it includes,
-    transitively, in first-seen order."""
+    """sha256 over a kernel source and every local device header (.cuh) it
+    includes, transitively, in first-seen order.  Headers of host-side
+    declarations (.h: launch functions and their parameter structs) do not
+    change a kernel's device code and are not followed."""
     seen, order = set(), []
 
     def walk(p):
@@ -75,7 +77,7 @@ def source_digest(path):
         seen.add(p)
         order.append(p)
         with open(p, "r", errors="replace") as f:
-            for inc in re.findall(r'^\s*#\s*include\s+"([^"]+)"', f.read(), re.M):
+            for inc in re.findall(r'^\s*#\s*include\s+"([^"]+\.cuh)"', f.read(), re.M):
                 walk(os.path.join(os.path.dirname(p), inc))
 
     walk(os.path.join(ROOT, path))
@@ -89,7 +91,7 @@ def source_digest(path):
 def measured_traffic(workload, kernel):
     """DRAM bytes (read + write) per launch from the ncu capture recorded in
     profiles/traffic.json, or None when there is none or the kernel's source
-    (its .cu file and the local headers it includes) has changed since."""
+    (its .cu file and the device headers it includes) has changed since."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f)[workload][kernel]

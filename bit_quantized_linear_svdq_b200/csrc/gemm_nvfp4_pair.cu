@@ -153,31 +153,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // The peer signals this CTA's barriers only after both have initialized them.
   cluster_sync();
-  // The weights (library-owned, written once at create time, which
-  // synchronizes) do not depend on the previous kernel: the first tile's
-  // first stages of weight codes and scale atoms start streaming now, while
-  // that kernel (the activation quantizer) may still be running.  The stage
-  // barriers are armed with the whole stage; the activation half follows in
-  // the producer loop.
-  const int npre = pair < num_tiles ? min(kStages, p.k_tiles) : 0;
-  if (tid == 0 && npre > 0) {
-    const int mt = pair % p.m_tiles, nt = pair / p.m_tiles;
-    const bool has_rows = 2 * mt + (int)rank < p.m_tiles128;
-    const int nrow0 = nt * BN + (BN / 2) * (int)rank;
-    prefetch_tmap(&tm_b);
-    for (int i = 0; i < npre; ++i) {
-      uint8_t* st = stages + i * kStageBytes;
-      const uint32_t fb = smem_u32(&full[i]);
-      if (leader) mbar_arrive_expect_tx(fb, 2u * (kABytes + kBBytes));
-      tma_load_2d_pair(smem_u32(st + kABytes), &tm_b, fb, i * kKTileBytes, nrow0);
-      const uint32_t sb = smem_u32(&sf_ld[i]);
-      mbar_arrive_expect_tx(sb, (uint32_t)((has_rows ? kSfaBytes : 0) + kSfbBytes));
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-        bulk_load(smem_u32(st + kABytes + kBBytes + kSfaBytes + h * (kSfbBytes / 2)),
-                  p.sfb + ((size_t)(2 * nt + h) * p.ka_pad + (size_t)i * kAtoms) * kSfAtomBytes, kSfbBytes / 2, sb);
-    }
-  }
   // Everything above overlaps the previous kernel's tail (programmatic
   // dependent launch); nothing below runs before it has completed.
   griddep_wait();
@@ -195,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       prefetch_tmap(&tm_a);
-      if (npre == 0) prefetch_tmap(&tm_b);
+      prefetch_tmap(&tm_b);
       prefetch_tmap(&tm_l);
       prefetch_tmap(&tm_pu);
       int g = 0, it = 0;
@@ -214,24 +189,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t* st = stages + s * kStageBytes;
           const uint32_t fb = smem_u32(&full[s]);
-          const uint32_t sb = smem_u32(&sf_ld[s]);
-          const bool pre = g < npre;              // armed, weight half in flight since the prologue
-          if (leader && !pre) mbar_arrive_expect_tx(fb, 2u * (kABytes + kBBytes));
+          if (leader) mbar_arrive_expect_tx(fb, 2u * (kABytes + kBBytes));
           tma_load_2d_pair(smem_u32(st), &tm_a, fb, kt * kKTileBytes, mrow0);
-          if (!pre) {
-            tma_load_2d_pair(smem_u32(st + kABytes), &tm_b, fb, kt * kKTileBytes, nrow0);
-            mbar_arrive_expect_tx(sb, (uint32_t)((has_rows ? kSfaBytes : 0) + kSfbBytes));
-          }
+          tma_load_2d_pair(smem_u32(st + kABytes), &tm_b, fb, kt * kKTileBytes, nrow0);
+          const uint32_t sb = smem_u32(&sf_ld[s]);
+          mbar_arrive_expect_tx(sb, (uint32_t)((has_rows ? kSfaBytes : 0) + kSfbBytes));
           if (has_rows)
             bulk_load(smem_u32(st + kABytes + kBBytes),
                       p.sfa + ((size_t)mt128 * p.ka_pad + (size_t)kt * kAtoms) * kSfAtomBytes, kSfaBytes, sb);
-          if (!pre) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-              bulk_load(smem_u32(st + kABytes + kBBytes + kSfaBytes + h * (kSfbBytes / 2)),
-                        p.sfb + ((size_t)(2 * nt + h) * p.ka_pad + (size_t)kt * kAtoms) * kSfAtomBytes,
-                        kSfbBytes / 2, sb);
-          }
+          for (int h = 0; h < 2; ++h)
+            bulk_load(smem_u32(st + kABytes + kBBytes + kSfaBytes + h * (kSfbBytes / 2)),
+                      p.sfb + ((size_t)(2 * nt + h) * p.ka_pad + (size_t)kt * kAtoms) * kSfAtomBytes, kSfbBytes / 2,
+                      sb);
           issued = g + 1;
           if (kt == p.k_tiles - 1) {
             // This CTA's L rows and proj_up' half, read after the K loop.
