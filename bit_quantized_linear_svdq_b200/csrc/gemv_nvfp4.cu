@@ -8,7 +8,8 @@
 // most eight multiply-adds, so the time is the weight read from HBM and the
 // kernel is a coalesced stream, not a tensor-core tile loop.
 //
-// Decomposition.  One CTA of 16 warps per SM; warp w of the grid owns weight
+// Decomposition.  One CTA of 16 warps per SM, on all but 8 SMs (left to the
+// quantizer that runs before it); warp w of the grid owns weight
 // rows w, w + W, w + 2W, ... (W = warps in the grid), two at a time.  Lane l
 // reads 16-byte pieces l, l + 32, ... of a row (32 FP4 codes = two scale
 // blocks each), so every load instruction of a warp covers 512 contiguous
@@ -43,6 +44,10 @@ namespace svdq {
 namespace {
 
 constexpr int kWarps = 16, kThreads = 32 * kWarps;
+// SMs left to the kernel before this one (the activation quantizer, whose K
+// split for at most four rows is one cluster of up to 8 CTAs), so that every
+// CTA of this kernel can start, and request its weights, while it runs.
+constexpr int kReserveSms = 8;
 constexpr int kPieces = 4;                 // 16-byte pieces per lane per row per pass (4096 K elements)
 constexpr int kPass = 32 * kPieces;        // pieces per row per pass
 
@@ -273,7 +278,7 @@ cudaError_t launch_gemv_nvfp4(const GemvLaunch& L, cudaStream_t stream) {
   p.K = L.K;
   p.Kp = L.Kp;
   p.R = L.R;
-  const int grid = std::max(1, std::min(L.num_sms, (L.N + kWarps - 1) / kWarps));
+  const int grid = std::max(1, std::min(L.num_sms - kReserveSms, (L.N + kWarps - 1) / kWarps));
   const size_t smem = gemv_smem_bytes(L.M, L.Kp, L.R);
   if (L.M == 1) return launch_mt<1>(p, grid, smem, stream);
   if (L.M == 2) return launch_mt<2>(p, grid, smem, stream);

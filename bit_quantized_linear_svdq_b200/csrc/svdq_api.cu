@@ -18,7 +18,7 @@ struct svdq_linear {
   int device;
   int K, N, R, Kp, ka_pad, k_tiles, rotate_block;
   uint8_t* qw;            // (N, Kp/2) packed E2M1, rows zero-padded to Kp
-  uint8_t* sfb;           // weight scale tiles: ceil(N/128) x ka_pad replicated atoms of 2 KB
+  uint8_t* sfb;           // weight scale tiles: (ceil(N/128) rounded up to even) x ka_pad atoms of 512 B
   uint8_t* sfr;           // (N, Kp/16) the same scales row-major, zero beyond K/16 (few-row CUDA-core product)
   __nv_bfloat16* pdT;     // proj_down^T (R, Kp), zero-padded
   __nv_bfloat16* pu;      // proj_up (N, R)
