@@ -44,7 +44,12 @@ plainest one the rest of the text supports):
 * y = wcscales[n] * wtscale * (Q(x_hat) Q(W)^T)[m, n] + (x_hat proj_down proj_up^T)[m, n].
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
-(page examples, closed forms, library routines, brute force, invariants).
+(page examples, closed forms, library routines, brute force, invariants).  The
+layer's composition -- divide by smooth_factor, then rotate, and the same x_hat
+in both branches -- is pinned by a hand-derived case with non-unit smoothing
+factors, by exact recovery of an on-grid x_hat through smoothing and a 4- or
+16-block rotation, and by the rotation identity y = (x R^T)(R W) through the
+rank-R branch and through the dense main product at block 128.
 """
 from __future__ import annotations
 

@@ -376,6 +376,51 @@ def test_hand_case_k32():
     np.testing.assert_array_equal(y[0], g["y"])
 
 
+def _hand_case_smooth():
+    g = _golden("hand_case_smooth_k32.json")
+
+    class C:
+        pass
+
+    ck = C()
+    M, K, N, R = (g["shape"][k] for k in ("M", "K", "N", "R"))
+    x = np.zeros((M, K))
+    for e in g["x_nonzero"]:
+        x[0, e["k"]] = e["value"]
+    ck.x = _bf16_bits(x)
+    lam = np.ones(K)
+    for e in g["smooth_factor_non_unit"]:
+        lam[e["k"]] = e["value"]
+    ck.smooth_factor = _bf16_bits(lam)
+    ck.qweight = np.zeros((N, K // 2), np.uint8)
+    for e in g["qweight_nonzero_bytes"]:
+        ck.qweight[e["n"], e["byte_index"]] = e["value"]
+    ck.wscales = np.full((K // 16, N), O.e4m3_encode_rne_satfinite(np.float32(g["wscales_all"])), np.uint8)
+    pd = np.zeros((K, R))
+    for e in g["proj_down_nonzero"]:
+        pd[e["k"], e["r"]] = e["value"]
+    ck.proj_down = _bf16_bits(pd)
+    ck.proj_up = _bf16_bits(g["proj_up"])
+    ck.wcscales = _bf16_bits(g["wcscales"])
+    ck.wtscale = _bf16_bits([g["wtscale"]])
+    ck.rotate_block = 0
+    return g, ck
+
+
+def test_hand_case_smooth_factor():
+    # [svdq] Checkpoint contract (smooth_factor): x_hat = x / smooth_factor
+    # feeds both the quantizer and the rank-R branch.  Every number in the
+    # fixture is derived by hand; unsmoothed or multiplied inputs, or a rank-R
+    # branch fed with x instead of x_hat, all change y.
+    g, ck = _hand_case_smooth()
+    codes, scales, xh = O.quantize_act(ck.x, ck.smooth_factor, 0)
+    np.testing.assert_array_equal(scales[0], g["act_scale_bytes"])
+    np.testing.assert_array_equal(codes[0], g["act_code_bytes"])
+    np.testing.assert_array_equal(O.lowrank_down(xh, ck.proj_down)[0], g["lowrank"])
+    y = O.linear_forward(ck)
+    np.testing.assert_array_equal(y[0], g["y"])
+
+
 def _grid_checkpoint(seed, M=3, K=64, N=5, R=4):
     """Activations whose every 16-block already lies on the NVFP4 grid (with a
     +-6s entry), smooth = 1, no rotation."""
@@ -464,6 +509,135 @@ def test_rotated_weight_quantizer_roundtrip():
     back = O.rotate_rows_f64(Wq, 128)
     rel = np.linalg.norm(back - O.bf16_to_f32(_bf16_bits(W))) / np.linalg.norm(W)
     assert rel < 0.2          # 4-bit with coarse (subnormal) e4m3 scales
+
+
+# ---------------------------------------------------------------- composition: smooth, then rotate, one x_hat for both branches
+
+def _rotation_matrix(K, block):
+    """Dense blockdiag(H_block / sqrt(block)) (K, K) from the Sylvester recursion."""
+    H = O.sylvester_hadamard(block) / np.sqrt(block)
+    R = np.zeros((K, K))
+    for b in range(K // block):
+        R[b * block:(b + 1) * block, b * block:(b + 1) * block] = H
+    return R
+
+
+@pytest.mark.parametrize("block", [4, 16])
+def test_exact_recovery_with_smoothing_and_rotation(block):
+    # [rot] 2.1 with [svdq] smooth_factor: pick the quantized target x_hat on
+    # the NVFP4 grid (power-of-two scales, a +-6s entry per block), then build
+    # the layer input that smoothing followed by rotation maps onto it:
+    # x_hat = (x / lam) R^T  <=>  x = (x_hat R) * lam  (R symmetric, R R = I).
+    # Blocks 4 and 16 normalise by 1/2 and 1/4, and lam holds powers of two,
+    # so every step is exact and y must equal the closed form exactly.  Rotating
+    # before smoothing, or feeding x (not x_hat) to the rank-R branch, breaks it.
+    rng = np.random.default_rng(20 + block)
+    M, K, N, R = 3, 64, 5, 4
+    xh = np.zeros((M, K))
+    for m in range(M):
+        for b in range(K // 16):
+            s = 2.0 ** int(rng.integers(-3, 3))
+            c = rng.integers(0, 16, 16)
+            c[rng.integers(0, 16)] = 7 if rng.random() < 0.5 else 15
+            xh[m, b * 16:(b + 1) * 16] = O.e2m1_decode(c) * s
+    lam = 2.0 ** rng.integers(-1, 3, K).astype(np.float64)
+    Rm = _rotation_matrix(K, block)
+    x = (xh @ Rm) * lam[None, :]
+
+    class C:
+        pass
+
+    ck = C()
+    ck.x = _bf16_bits(x)
+    assert np.array_equal(O.bf16_to_f32(ck.x).astype(np.float64), x)        # representable
+    ck.smooth_factor = _bf16_bits(lam)
+    ck.qweight = rng.integers(0, 256, (N, K // 2)).astype(np.uint8)
+    ck.wscales = O.e4m3_encode_rne_satfinite(rng.uniform(0.01, 0.1, (K // 16, N)).astype(np.float32))
+    ck.proj_down = _bf16_bits(rng.standard_normal((K, R)) * 0.02)
+    ck.proj_up = _bf16_bits(rng.standard_normal((N, R)) * 0.02)
+    ck.wcscales = _bf16_bits(rng.uniform(0.8, 1.2, N))
+    ck.wtscale = _bf16_bits([0.5])
+    ck.rotate_block = block
+    codes, scales, xh_o = O.quantize_act(ck.x, ck.smooth_factor, block)
+    np.testing.assert_array_equal(xh_o.astype(np.float64), xh)
+    np.testing.assert_array_equal(O.dequantize_nvfp4(codes, scales), xh)
+    W = O.dequantize_weight(ck.qweight, ck.wscales)
+    alpha = O.bf16_to_f32(ck.wcscales).astype(np.float64) * 0.5
+    pd = O.bf16_to_f32(ck.proj_down).astype(np.float64)
+    pu = O.bf16_to_f32(ck.proj_up).astype(np.float64)
+    y_exact = alpha * (xh @ W.T) + (xh @ pd) @ pu.T
+    np.testing.assert_allclose(O.linear_forward(ck), y_exact, rtol=1e-13, atol=1e-13)
+
+
+def _random_layer_input(rng, M, K):
+    x = rng.standard_normal((M, K)) * 2.0
+    x[:, rng.choice(K, 3, replace=False)] *= 30.0
+    lam = rng.uniform(0.5, 2.0, K)
+    return _bf16_bits(x), _bf16_bits(lam)
+
+
+def test_rotation_identity_through_rank_r_branch():
+    # [rot] 2.1: (x R^T)(R P) = x P.  With every weight code zero, y is the
+    # rank-R branch alone, so the 128-block rotated layer with proj_down' =
+    # bf16(R proj_down) must give the unrotated layer's y.  The two differ only
+    # by the bf16 rounding of proj_down' (2^-9 relative per entry) and the fp32
+    # rounding of x_hat (at most a few 2^-24 relative per butterfly stage);
+    # the bound below is that, entry by entry.  Rotating before smoothing, or
+    # a rank-R branch fed with x, misses it by orders of magnitude.
+    rng = np.random.default_rng(41)
+    M, K, N, R = 4, 256, 6, 3
+    x_bits, lam_bits = _random_layer_input(rng, M, K)
+    pd = O.bf16_to_f32(_bf16_bits(rng.standard_normal((K, R)) * 0.02)).astype(np.float64)
+    Rm = _rotation_matrix(K, 128)
+    pd_rot_bits = _bf16_bits(Rm @ pd)
+
+    class C:
+        pass
+
+    def layer(block, pd_bits):
+        ck = C()
+        ck.x, ck.smooth_factor = x_bits, lam_bits
+        ck.qweight = np.zeros((N, K // 2), np.uint8)
+        ck.wscales = O.e4m3_encode_rne_satfinite(np.full((K // 16, N), 0.05, np.float32))
+        ck.proj_down = pd_bits
+        ck.proj_up = _bf16_bits(rng_pu)
+        ck.wcscales = _bf16_bits(np.ones(N))
+        ck.wtscale = _bf16_bits([1.0])
+        ck.rotate_block = block
+        return O.linear_forward(ck)
+
+    rng_pu = rng.standard_normal((N, R)) * 0.02
+    y_plain = layer(0, _bf16_bits(pd))
+    y_rot = layer(128, pd_rot_bits)
+    xs = np.abs(O.bf16_to_f32(x_bits).astype(np.float64) / O.bf16_to_f32(lam_bits).astype(np.float64))
+    rpd = Rm @ pd
+    pu = np.abs(O.bf16_to_f32(_bf16_bits(rng_pu)).astype(np.float64))
+    xh_rot = np.abs(O.smooth_and_rotate(x_bits, lam_bits, 128).astype(np.float64))
+    xr = xs @ np.abs(Rm)                             # l1 bound on a rotated entry's partial sums
+    bound_L = xh_rot @ (2.0 ** -9 * np.abs(rpd)) + 16 * 2.0 ** -24 * (xr @ np.abs(rpd) + xs @ np.abs(pd))
+    bound = bound_L @ pu.T
+    assert np.all(np.abs(y_rot - y_plain) <= bound), np.max(np.abs(y_rot - y_plain) / bound)
+    assert np.max(np.abs(y_plain)) > 10 * np.max(bound)      # the check is not vacuous
+
+
+def test_rotation_identity_through_main_product_dense():
+    # [rot] 2.1 on the main product before quantization: with W' = W R^T (the
+    # checkpoint's (N, K) rows rotated), x_hat_rot W'^T = x_hat W^T, where
+    # x_hat_rot is the oracle's smoothed-then-rotated activation.  Exact up to
+    # the fp32 rounding of x_hat; smoothing after rotating misses it.
+    rng = np.random.default_rng(43)
+    M, K, N = 5, 384, 7
+    x_bits, lam_bits = _random_layer_input(rng, M, K)
+    W = rng.standard_normal((N, K))
+    xh0 = O.smooth_and_rotate(x_bits, lam_bits, 0).astype(np.float64)
+    xh1 = O.smooth_and_rotate(x_bits, lam_bits, 128).astype(np.float64)
+    Wr = O.rotate_rows_f64(W, 128)
+    y0 = xh0 @ W.T
+    y1 = xh1 @ Wr.T
+    scale = np.abs(xh0) @ np.abs(W).T
+    assert np.all(np.abs(y1 - y0) <= 2.0 ** -19 * scale + 1e-12)
+    # the exact real x_hat R^T agrees with the fp32 one to fp32 rounding
+    np.testing.assert_allclose(xh1, O.rotate_rows_f64(xh0, 128), rtol=0, atol=2.0 ** -20 * np.abs(xh0).max())
 
 
 # ---------------------------------------------------------------- [rot] section 3.1: the standalone transform
