@@ -65,15 +65,21 @@ def build(verbose: bool = False, force: bool = False) -> str:
     objdir = os.path.join(LIBDIR, "obj")
     os.makedirs(objdir, exist_ok=True)
     nvcc = _nvcc()
-    objs = []
+    objs, cmds = [], []
     for src in srcs:
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [nvcc, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
+        cmds.append(cmd)
         objs.append(obj)
+    # One nvcc process per source, as many at once as there are cores.
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as pool:
+        for r in list(pool.map(lambda c: subprocess.run(c, capture_output=not verbose, text=True), cmds)):
+            if r.returncode != 0:
+                raise RuntimeError("nvcc failed: " + " ".join(r.args) + "\n" + (r.stderr or "") + (r.stdout or ""))
     tmp = LIB + ".tmp"
     cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs, "-lcudart_static",
            "-Xcompiler", "-fvisibility=hidden"]

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -20,11 +21,10 @@ struct svdq_linear {
   uint8_t* qw;            // (N, Kp/2) packed E2M1, rows zero-padded to Kp
   uint8_t* sfb;           // weight scale tiles: (ceil(N/128) rounded up to even) x ka_pad atoms of 512 B
   uint8_t* sfr;           // (N, Kp/16) the same scales row-major, zero beyond K/16 (few-row CUDA-core product)
-  __nv_bfloat16* pdT;     // proj_down^T (R, Kp), zero-padded
+  __nv_bfloat16* pdT;     // P^T (R, Kp), P = diag(1/smooth) R^T proj_down in bf16, zero-padded
   __nv_bfloat16* pu;      // proj_up (N, R)
-  float4* lam4;           // (Kp/2) {-s_k, -s_k+1, 1/s_k, 1/s_k+1} per channel pair, padded with s = 1
-  float4* lam4_neg;       // (Kp/2) the same operands for dividing by -s_k
-  bool lam_positive;      // every smooth factor is positive
+  float4* lamq;           // (Kp/2) {yh_k, yh_k+1, yl_k, yl_k+1}: RZ(1/s) and RN(1/s - RZ(1/s)), padded with s = 1
+  float* lamf;            // (Kp) smooth factors as fp32, padded with 1
   float* alpha;           // (roundup(N, 128)) wcscales * wtscale, zero-padded
   __nv_bfloat16* pu_fold; // proj_up' = bf16(proj_up / alpha) (N, R); proj_up where alpha = 0
   float* alpha_fold;      // (roundup(N, 256)) alpha, or 1 where alpha = 0
@@ -126,34 +126,73 @@ __global__ void repack_weight_scales(const uint8_t* __restrict__ wscales, const 
   }
 }
 
-__global__ void transpose_proj_down(const __nv_bfloat16* __restrict__ pd, __nv_bfloat16* __restrict__ pdT, int K,
-                                    int R, int Kp) {
+// P^T (R, Kp) for the quantizer's down-projection, P = diag(1/s) R^T proj_down:
+// x_hat proj_down = ((x / s) R^T) proj_down = x P, so the tensor core can read
+// the raw x tile.  R = blockdiag(H_128 / sqrt(128)) (symmetric) or the
+// identity.  Each entry in double precision (the rotation sum is exact in
+// double for bf16 inputs up to rounding at 2^-53), then rounded to bf16.
+// Padding channels are zero.  bad bit 32: an entry overflows bf16.
+__global__ void prepare_proj_down(const __nv_bfloat16* __restrict__ pd, const __nv_bfloat16* __restrict__ sf,
+                                  __nv_bfloat16* __restrict__ pdT, int K, int R, int Kp, int rot, unsigned* bad) {
   const long long total = (long long)R * Kp;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
     const int r = (int)(i / Kp), k = (int)(i % Kp);
-    pdT[i] = k < K ? pd[(size_t)k * R + r] : __float2bfloat16_rn(0.0f);
+    if (k >= K) {
+      pdT[i] = __float2bfloat16_rn(0.0f);
+      continue;
+    }
+    double acc;
+    if (rot) {
+      // (R proj_down)[k, r] = sum_t H[k % 128][t] proj_down[128 * (k / 128) + t, r] / sqrt(128),
+      // H[a][b] = (-1)^popcount(a & b) (Sylvester).
+      const int kb = k & ~127, kr = k & 127;
+      acc = 0.0;
+      for (int t = 0; t < 128; ++t) {
+        const double v = (double)__bfloat162float(pd[(size_t)(kb + t) * R + r]);
+        acc += (__popc(kr & t) & 1) ? -v : v;
+      }
+      acc /= sqrt(128.0);
+    } else {
+      acc = (double)__bfloat162float(pd[(size_t)k * R + r]);
+    }
+    const double val = acc / (double)__bfloat162float(sf[k]);
+    const __nv_bfloat16 q = __float2bfloat16_rn(__double2float_rn(val));
+    if (!isfinite(__bfloat162float(q))) atomicOr(bad, 32u);
+    pdT[i] = q;
   }
 }
 
-// Per channel pair (k, k+1): {-s_k, -s_k+1, RN(1/s_k), RN(1/s_k+1)} and its
-// negation, the operands of the quantizer's two-lane correctly rounded
-// division by s or by -s; padding channels get s = 1.  Stored in the
-// quantizer's bank-conflict-free order (svdq::lam_slot).  bad bit 2: a zero or
-// non-finite factor; bit 4: a negative one.
-__global__ void prepare_smooth(const __nv_bfloat16* __restrict__ sf, float4* __restrict__ lam4,
-                               float4* __restrict__ lam4_neg, int K, int Kp, unsigned* bad) {
+// Per channel pair (k, k+1): the reciprocal pairs {yh_k, yh_k+1, yl_k, yl_k+1}
+// with yh = RZ(1/s) and yl = RN(1/s - yh) (sign of yh), from which the
+// quantizer forms the correctly rounded x / s as RN(x*yh + RN(x*yl)); stored in
+// its bank-conflict-free order (svdq::lam_slot).  Also the factors themselves
+// as fp32 (the IEEE path).  Padding channels get s = 1.  bad bit 2: a zero or
+// non-finite factor; bit 16: a factor outside the magnitudes [2^-126, 2^117)
+// for which that division is exact.
+__global__ void prepare_smooth(const __nv_bfloat16* __restrict__ sf, float4* __restrict__ lamq, float* __restrict__ lamf,
+                               int K, int Kp, unsigned* bad) {
   for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < Kp / 2; j += gridDim.x * blockDim.x) {
-    float l0 = 1.0f, l1 = 1.0f;
+    float l[2] = {1.0f, 1.0f};
     if (2 * j < K) {                 // K is even, so channel 2j+1 exists too
-      l0 = __bfloat162float(sf[2 * j]);
-      l1 = __bfloat162float(sf[2 * j + 1]);
-      if (!(isfinite(l0) && l0 != 0.0f && isfinite(l1) && l1 != 0.0f)) atomicOr(bad, 2u);
-      if (l0 < 0.0f || l1 < 0.0f) atomicOr(bad, 4u);
+      l[0] = __bfloat162float(sf[2 * j]);
+      l[1] = __bfloat162float(sf[2 * j + 1]);
     }
-    const float r0 = __frcp_rn(l0), r1 = __frcp_rn(l1);
-    const int o = svdq::lam_slot(j);
-    lam4[o] = make_float4(-l0, -l1, r0, r1);
-    lam4_neg[o] = make_float4(l0, l1, -r0, -r1);
+    float yh[2], yl[2];
+    for (int c = 0; c < 2; ++c) {
+      const float a = fabsf(l[c]);
+      if (!(isfinite(l[c]) && l[c] != 0.0f)) {
+        atomicOr(bad, 2u);
+        l[c] = 1.0f;
+      } else if (a < 0x1p-126f || a >= 0x1p117f) {
+        atomicOr(bad, 16u);
+      }
+      const double inv = 1.0 / (double)l[c];
+      yh[c] = __double2float_rz(inv);
+      yl[c] = copysignf(fabsf(__double2float_rn(inv - (double)yh[c])), yh[c]);
+    }
+    lamq[svdq::lam_slot(j)] = make_float4(yh[0], yh[1], yl[0], yl[1]);
+    lamf[2 * j] = l[0];
+    lamf[2 * j + 1] = l[1];
   }
 }
 
@@ -222,8 +261,8 @@ void free_handle(svdq_linear* h) {
   cudaFree(h->sfr);
   cudaFree(h->pdT);
   cudaFree(h->pu);
-  cudaFree(h->lam4);
-  cudaFree(h->lam4_neg);
+  cudaFree(h->lamq);
+  cudaFree(h->lamf);
   cudaFree(h->alpha);
   cudaFree(h->pu_fold);
   cudaFree(h->alpha_fold);
@@ -329,8 +368,8 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
   CREATE_CUDA(cudaMalloc(&h->sfr, (size_t)d->N * (h->Kp / 16)));
   CREATE_CUDA(cudaMalloc(&h->pdT, (size_t)d->R * h->Kp * 2));
   CREATE_CUDA(cudaMalloc(&h->pu, (size_t)d->N * d->R * 2));
-  CREATE_CUDA(cudaMalloc(&h->lam4, (size_t)(h->Kp / 2) * sizeof(float4)));
-  CREATE_CUDA(cudaMalloc(&h->lam4_neg, (size_t)(h->Kp / 2) * sizeof(float4)));
+  CREATE_CUDA(cudaMalloc(&h->lamq, (size_t)(h->Kp / 2) * sizeof(float4)));
+  CREATE_CUDA(cudaMalloc(&h->lamf, (size_t)h->Kp * sizeof(float)));
   CREATE_CUDA(cudaMalloc(&h->alpha, (size_t)Npad * sizeof(float)));
   CREATE_CUDA(cudaMalloc(&h->pu_fold, (size_t)d->N * d->R * 2));
   CREATE_CUDA(cudaMalloc(&h->alpha_fold, (size_t)Npad256 * sizeof(float)));
@@ -358,24 +397,27 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
       static_cast<const uint8_t*>(d->wscales), h->alpha, h->sfb, h->sfr, d->K / 16, d->N, h->ka_pad, h->Kp / 16,
       h->err + 1);
   CREATE_CUDA(cudaGetLastError());
-  transpose_proj_down<<<grid_for((long long)d->R * h->Kp), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(d->proj_down), h->pdT, d->K, d->R, h->Kp);
+  prepare_smooth<<<grid_for(h->Kp / 2), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(d->smooth_factor), h->lamq,
+                                                           h->lamf, d->K, h->Kp, h->err + 1);
+  CREATE_CUDA(cudaGetLastError());
+  prepare_proj_down<<<grid_for((long long)d->R * h->Kp), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(d->proj_down), static_cast<const __nv_bfloat16*>(d->smooth_factor), h->pdT,
+      d->K, d->R, h->Kp, d->rotate_block == 128, h->err + 1);
   CREATE_CUDA(cudaGetLastError());
   CREATE_CUDA(cudaMemcpyAsync(h->pu, d->proj_up, (size_t)d->N * d->R * 2, cudaMemcpyDeviceToDevice, stream));
-  prepare_smooth<<<grid_for(h->Kp / 2), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(d->smooth_factor), h->lam4,
-                                                           h->lam4_neg, d->K, h->Kp, h->err + 1);
-  CREATE_CUDA(cudaGetLastError());
   fold_alpha<<<grid_for((long long)Npad256 * d->R), 256, 0, stream>>>(h->pu, h->alpha, h->pu_fold, h->alpha_fold,
                                                                       d->N, d->R, Npad256, h->err + 1);
   CREATE_CUDA(cudaGetLastError());
   unsigned bad = 0;
   CREATE_CUDA(cudaMemcpyAsync(&bad, h->err + 1, sizeof(unsigned), cudaMemcpyDeviceToHost, stream));
   CREATE_CUDA(cudaStreamSynchronize(stream));
-  if (bad & 3u) {
-    g_last_error = (bad & 1u) ? "wscales holds an e4m3 NaN" : "smooth_factor holds a zero or non-finite value";
+  if (bad & (1u | 2u | 16u | 32u)) {
+    g_last_error = (bad & 1u)    ? "wscales holds an e4m3 NaN"
+                   : (bad & 2u)  ? "smooth_factor holds a zero or non-finite value"
+                   : (bad & 16u) ? "smooth_factor holds a magnitude outside [2^-126, 2^117)"
+                                 : "proj_down / smooth_factor overflows bf16";
     return fail(SVDQ_ERR_INVALID_ARG);
   }
-  h->lam_positive = (bad & 4u) == 0;
   {
     // 128 x 256 tiles unless alpha cannot be folded, R > 32, or the
     // environment asks for the 128 x 128 GEMM (SVDQ_GEMM_TILE_N=128).
@@ -454,9 +496,8 @@ svdq_status svdq_quantize_act(const svdq_linear* h, const void* x, int M, void* 
     return s;
   q.tm_pdT = h->tm_pdT;
   q.tm_codes = q.tm_x;   // unused: the public layout is written directly
-  q.lam4 = h->lam4;
-  q.lam4_neg = h->lam4_neg;
-  q.lam_positive = h->lam_positive;
+  q.lamq = h->lamq;
+  q.lamf = h->lamf;
   q.codes = static_cast<uint8_t*>(codes);
   q.scales = static_cast<uint8_t*>(scales);
   q.lowrank = lowrank;
@@ -496,9 +537,8 @@ svdq_status forward_quantize(const svdq_linear* h, const void* x, int M, void* w
   if ((s = make_tmap(&q.tm_codes, ws + w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->Kp / 2, M, h->Kp / 2, 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_NONE)) != SVDQ_OK)
     return s;
-  q.lam4 = h->lam4;
-  q.lam4_neg = h->lam4_neg;
-  q.lam_positive = h->lam_positive;
+  q.lamq = h->lamq;
+  q.lamf = h->lamf;
   q.codes = ws + w.codes;
   q.scales = ws + w.sfa;
   q.lowrank = ws + w.lr;

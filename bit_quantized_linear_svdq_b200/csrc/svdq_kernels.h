@@ -9,14 +9,15 @@
 namespace svdq {
 
 // Fused activation quantizer: x_hat = x / smooth (optionally block-Hadamard
-// rotated), NVFP4 codes + e4m3 scales, and L = x_hat @ proj_down.
+// rotated), NVFP4 codes + e4m3 scales, and L = x_hat @ proj_down computed as
+// x @ P with P = diag(1/smooth) R^T proj_down.
 struct QuantLaunch {
   CUtensorMap tm_x;         // x bf16 (M, K): box {64, 128}, 128B swizzle
-  CUtensorMap tm_pdT;       // proj_down^T bf16 (R, Kp): box {64, R}, 128B swizzle
+  CUtensorMap tm_pdT;       // P^T bf16 (R, Kp): box {64, R}, 128B swizzle
   CUtensorMap tm_codes;     // tiled_scales only: codes u8 (M, Kp/2): box {64, 128}, no swizzle (TMA store)
-  const void* lam4;         // float4 (Kp/2): {-s_k, -s_k+1, 1/s_k, 1/s_k+1} per channel pair, padded with s = 1
-  const void* lam4_neg;     // float4 (Kp/2): {s_k, s_k+1, -1/s_k, -1/s_k+1} (dividing by -smooth)
-  bool lam_positive;        // every smooth factor > 0: the negated layout may be used
+  const void* lamq;         // float4 (Kp/2): {yh_k, yh_k+1, yl_k, yl_k+1} per channel pair (yh = RZ(1/s),
+                            // yl = RN(1/s - yh) with yh's sign), lam_slot order, padded with s = 1
+  const float* lamf;        // (Kp) smooth factors as fp32, padded with 1 (IEEE path)
   uint8_t* codes;           // packed codes, row pitch codes_pitch bytes
   uint8_t* scales;          // row-major (pitch scales_pitch) or tensor-core tiles
   void* lowrank;            // bf16 (M, R) or nullptr

@@ -13,7 +13,11 @@
 // the process exits.  Host code never takes its address directly (on the host
 // the symbol is only a stand-in); the device address comes from
 // cudaGetSymbolAddress, looked up once per device by the first call made with
-// that device current, and cached.
+// that device current, and cached together with the identity of the device's
+// context.  A cudaDeviceReset replaces that context (and reloads the module,
+// so the array may move): the next call sees a new context id and looks the
+// address up again instead of writing through a stale pointer.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -30,18 +34,50 @@ static __device__ __align__(256) uint8_t g_scratch[kScratchBytes];
 
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices];
+unsigned long long g_scratch_ctx[kMaxDevices];   // context id the cached address belongs to
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Id of the context current on this thread (0 when none is, or the driver
+// calls are unavailable).  Driver entry points come through the runtime.
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 // Device address of this device's copy of the array; NULL (and the CUDA error
-// cleared) if the lookup fails.
+// cleared) if the lookup fails.  Looked up on the first call for the device
+// and again whenever the device's current context is not the one the cached
+// address came from.
 void* scratch_on(int dev) {
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
+  const unsigned long long ctx = current_ctx_id();
+  if (!g_scratch_addr[dev] || ctx == 0 || ctx != g_scratch_ctx[dev]) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_scratch) != cudaSuccess || !ptr) {
       cudaGetLastError();
+      g_scratch_addr[dev] = nullptr;
       return nullptr;
     }
     g_scratch_addr[dev] = ptr;
+    g_scratch_ctx[dev] = current_ctx_id();   // the lookup made the primary context current
   }
   return g_scratch_addr[dev];
 }

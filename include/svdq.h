@@ -29,9 +29,15 @@
  *    SVDQ_ERR_CUDA the CUDA error text is available from svdq_last_error().
  *  - The device must be compute capability 10.0 (B200, sm_100a); create()
  *    checks the current device.
- *  - A handle is used on the device that was current at create().  Calls on
- *    one handle from several host threads are safe (the handle is read-only
- *    after create) as long as their workspaces differ.
+ *  - A handle is used on the device that was current at create().  The calls
+ *    that take a caller workspace (svdq_quantize_act, svdq_linear_forward and
+ *    its two stages) may run on one handle from several host threads at once:
+ *    they only read the handle, so it is safe as long as their workspaces and
+ *    outputs differ.  Two calls are exceptions: svdq_linear_forward_host uses
+ *    copy streams and events owned by the handle, so its calls on one handle
+ *    must not overlap; svdq_linear_forward_noalloc shares one scratch array
+ *    per device among all its calls, so calls whose kernels can overlap on
+ *    the GPU race (see each declaration).
  */
 #ifndef SVDQ_H_
 #define SVDQ_H_
@@ -79,7 +85,7 @@ typedef struct {
   const void* wscales;        /* (K/16, N) float8_e4m3fn: wscales[k/16, n] scales W[n, k] */
   const void* proj_down;      /* (K, R)    bf16 */
   const void* proj_up;        /* (N, R)    bf16 */
-  const void* smooth_factor;  /* (K,)      bf16, finite and nonzero */
+  const void* smooth_factor;  /* (K,)      bf16, finite, magnitude in [2^-126, 2^117) */
   const void* wcscales;       /* (N,)      bf16, or NULL meaning all ones */
   const void* wtscale;        /* (1,)      bf16, or NULL meaning 1.0 */
 } svdq_linear_desc;
@@ -87,8 +93,14 @@ typedef struct {
 /*
  * svdq_linear_create -- validate the description and copy + repack the
  * weights into library-owned device memory (FP4 weight rows padded for TMA,
- * scale factors re-tiled into the tensor-core scale layout, proj_down
- * transposed, alpha[n] = wcscales[n] * wtscale precomputed in fp32).
+ * scale factors re-tiled into the tensor-core scale layout, the down-projection
+ * folded with the smoothing and the rotation as P = diag(1/smooth_factor) R^T
+ * proj_down in bf16 (so that x_hat proj_down = x P), reciprocal pairs of the
+ * smoothing factors for the exact division, alpha[n] = wcscales[n] * wtscale
+ * precomputed in fp32).  Returns SVDQ_ERR_INVALID_ARG for a wscales NaN, a
+ * smoothing factor that is zero, non-finite or of magnitude outside
+ * [2^-126, 2^117) (the range in which the quantizer's division is exact), or a
+ * P entry that overflows bf16; svdq_last_error() names which.
  * The source tensors may be freed once this returns: it synchronizes `stream`.
  * On success *out receives the handle; on failure *out is set to NULL.
  * Shape errors are reported here (the pages' fail-at-load convention,
@@ -109,8 +121,9 @@ SVDQ_API size_t svdq_workspace_bytes(const svdq_linear* h, int M);
  *   x       (M, K)    bf16, input
  *   codes   (M, K/2)  uint8 output: packed E2M1 codes, low nibble = even k
  *   scales  (M, K/16) uint8 output: e4m3 scale bytes, row-major
- *   lowrank (M, R)    bf16 output L = x_hat proj_down (fp32 accumulate of
- *                     bf16(x_hat) products), or NULL to skip writing it
+ *   lowrank (M, R)    bf16 output L = x_hat proj_down, computed as x P with
+ *                     P = bf16(diag(1/smooth_factor) R^T proj_down) (fp32
+ *                     accumulate on the tensor cores), or NULL to skip it
  * M == 0 is a no-op.  Pointers must be 16-byte aligned.
  */
 SVDQ_API svdq_status svdq_quantize_act(const svdq_linear* h, const void* x, int M,
@@ -179,7 +192,10 @@ SVDQ_API svdq_status svdq_linear_forward_host(const svdq_linear* h, const void* 
  * 14,000 rows at K = 3072, R = 32); use svdq_linear_forward for larger M.
  * The first call on each device (made with that device current) looks up the
  * array's device address and caches it; make that first call before any
- * stream capture begins.  The call itself allocates and frees nothing.
+ * stream capture begins.  The cache is tied to the device's context: after a
+ * cudaDeviceReset the next call finds a new context and looks the address up
+ * again (the array then starts over in the new context).  The call itself
+ * allocates and frees nothing.
  * Every call on a device -- any handle, thread or stream -- shares the one
  * array, which keeps the previous call's contents: calls whose kernels can
  * overlap on the GPU race and corrupt each other's results, so order them (one
