@@ -407,6 +407,32 @@ def run_ours(args, world, rank, local):
     t_ht = timed(g_ht)
     del g_ht, hsets
 
+    # The MXFP4 linear with a grouped Hadamard (the FP-Quant forward: fused
+    # group-32 rotation + MXFP4 quantizer, then the MXFP4 GEMM) on this
+    # layer's shape: seeded W ~ N(0, 0.02) quantized on the GPU, x ~ N(0, 1).
+    msets = []
+    for i in range(N_SETS):
+        w = (torch.randn((N, K), generator=gen, device="cuda") * 0.02).to(torch.bfloat16)
+        qw_m, ws_m = S.mxfp4_quantize(w, 32)
+        lay_m = S.MXFP4Linear(qw_m, ws_m, alpha=1.0, hadamard_group=32)
+        xm = torch.randn((M, K), generator=gen, device="cuda").to(torch.bfloat16)
+        ym = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        msets.append((lay_m, xm, ym, lay_m.workspace(M)))
+        del w, qw_m, ws_m
+
+    def mxf(i):
+        lay_m, xm, ym, wsm = msets[i % N_SETS]
+        S.svdq_mxfp4_forward(lay_m.handle, xm.data_ptr(), M, ym.data_ptr(), wsm.data_ptr(), stream)
+
+    g_mx = graph_calls(mxf)
+    t_mx = timed(g_mx)
+    del g_mx
+    for lay_m, *_ in msets:
+        if lay_m.device_status() != 0:
+            raise SystemExit("device error flag set in the MXFP4 forward")
+        lay_m.close()
+    del msets
+
     # End-to-end through the host-buffer C ABI call: H2D of x, forward, D2H of y, sync.
     layer, x, y, ws = sets[0]
     xh = x.cpu().pin_memory()
@@ -438,6 +464,7 @@ def run_ours(args, world, rank, local):
     us_g = t_gemm / args.steps * 1e6
     us_wq = t_wq / args.steps * 1e6
     us_ht = t_ht / args.steps * 1e6
+    us_mx = t_mx / args.steps * 1e6
     ht_bytes = 2.0 * 2 * M * HN
     wq_bytes = 2.0 * N * K + N * K / 2 + N * K / 16
     q_gbs = quant_bytes(M, K, R) / (us_q * 1e-6) / 1e9
@@ -457,6 +484,11 @@ def run_ours(args, world, rank, local):
                                "frac_of_hbm": ht_bytes / (us_ht * 1e-6) / 1e9 / pk["hbm_gbs"],
                                "traffic": measured_traffic(ck.name, "hadamard_transform"),
                                "note": f"standalone transform, in place on {M} x {HN} bf16"},
+        "mxfp4_forward": {"us": us_mx, "bound": "tensor", "algorithmic_flops": 2.0 * M * N * K,
+                          "achieved_tflops": 2.0 * M * N * K / (us_mx * 1e-6) / 1e12,
+                          "frac_of_fp4": 2.0 * M * N * K / (us_mx * 1e-6) / 1e12 / fp4_peak,
+                          "note": "FP-Quant forward on this layer's shape: group-32 Hadamard + MXFP4 quantizer, "
+                                  "then the MXFP4 GEMM (two launches), weights quantized on the GPU"},
         "gemm_nvfp4": {"us": us_g, "bound": gemm_bound, "variant": variant, "algorithmic_flops": g_flops,
                        "achieved_tflops": g_tf, "frac_of_fp4": g_tf / fp4_peak,
                        "algorithmic_bytes": gemm_bytes(M, K, N, R),

@@ -23,7 +23,10 @@ __all__ = [
     "svdq_linear_create", "svdq_linear_destroy", "svdq_workspace_bytes", "svdq_quantize_act",
     "svdq_linear_forward", "svdq_linear_forward_host", "svdq_linear_forward_quantize",
     "svdq_linear_forward_gemm", "svdq_linear_gemm_kernel", "svdq_device_status", "svdq_status_string",
-    "svdq_last_error", "svdq_version", "svdq_quantize_weight", "quantize_weight", "svdq_hadamard_transform", "hadamard_transform", "SVDQLinear", "STATUS",
+    "svdq_last_error", "svdq_version", "svdq_quantize_weight", "quantize_weight", "svdq_hadamard_transform",
+    "hadamard_transform", "SVDQLinear", "STATUS", "svdq_mxfp4_desc", "svdq_mxfp4_create", "svdq_mxfp4_destroy",
+    "svdq_mxfp4_workspace_bytes", "svdq_mxfp4_quantize", "svdq_mxfp4_forward", "svdq_mxfp4_device_status",
+    "mxfp4_quantize", "MXFP4Linear",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -55,6 +58,13 @@ class svdq_linear_desc(ctypes.Structure):
         ("proj_down", ctypes.c_void_p), ("proj_up", ctypes.c_void_p),
         ("smooth_factor", ctypes.c_void_p), ("wcscales", ctypes.c_void_p),
         ("wtscale", ctypes.c_void_p),
+    ]
+
+
+class svdq_mxfp4_desc(ctypes.Structure):
+    _fields_ = [
+        ("K", ctypes.c_int), ("N", ctypes.c_int), ("hadamard_group", ctypes.c_int),
+        ("qweight", ctypes.c_void_p), ("wscales", ctypes.c_void_p), ("alpha", ctypes.c_float),
     ]
 
 
@@ -93,6 +103,12 @@ def load_library() -> ctypes.CDLL:
         "svdq_version": (ci, []),
         "svdq_quantize_weight": (ci, [vp, ci, ci, ci, vp, vp, vp]),
         "svdq_hadamard_transform": (ci, [vp, ci, ci, ci, vp]),
+        "svdq_mxfp4_create": (ci, [ctypes.POINTER(vp), ctypes.POINTER(svdq_mxfp4_desc), vp]),
+        "svdq_mxfp4_destroy": (None, [vp]),
+        "svdq_mxfp4_workspace_bytes": (cs, [vp, ci]),
+        "svdq_mxfp4_quantize": (ci, [vp, ci, ci, ci, vp, vp, vp]),
+        "svdq_mxfp4_forward": (ci, [vp, vp, ci, vp, vp, vp]),
+        "svdq_mxfp4_device_status": (ci, [vp, ctypes.POINTER(ci)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -217,6 +233,100 @@ def hadamard_transform(x: torch.Tensor, inplace: bool = True, stream=None) -> to
     rows = y.numel() // n if n else 0
     svdq_hadamard_transform(y.data_ptr(), rows, n, 0 if y.dtype == torch.bfloat16 else 1, stream)
     return y
+
+
+def svdq_mxfp4_create(desc: "svdq_mxfp4_desc", stream=None) -> int:
+    h = ctypes.c_void_p()
+    _check(load_library().svdq_mxfp4_create(ctypes.byref(h), ctypes.byref(desc), _stream(stream)),
+           "svdq_mxfp4_create")
+    return h.value
+
+
+def svdq_mxfp4_destroy(handle: Optional[int]) -> None:
+    load_library().svdq_mxfp4_destroy(handle)
+
+
+def svdq_mxfp4_workspace_bytes(handle: int, M: int) -> int:
+    return load_library().svdq_mxfp4_workspace_bytes(handle, M)
+
+
+def svdq_mxfp4_quantize(x_ptr, M, K, hadamard_group, codes_ptr, scales_ptr, stream=None) -> None:
+    _check(load_library().svdq_mxfp4_quantize(x_ptr, M, K, hadamard_group, codes_ptr, scales_ptr, _stream(stream)),
+           "svdq_mxfp4_quantize")
+
+
+def svdq_mxfp4_forward(handle, x_ptr, M, y_ptr, workspace_ptr, stream=None) -> None:
+    _check(load_library().svdq_mxfp4_forward(handle, x_ptr, M, y_ptr, workspace_ptr, _stream(stream)),
+           "svdq_mxfp4_forward")
+
+
+def svdq_mxfp4_device_status(handle) -> int:
+    flags = ctypes.c_int(0)
+    st = load_library().svdq_mxfp4_device_status(handle, ctypes.byref(flags))
+    if st not in (0, 6):
+        raise SvdqError(st, "svdq_mxfp4_device_status")
+    return flags.value
+
+
+def mxfp4_quantize(x: torch.Tensor, hadamard_group: int = 32, stream=None):
+    """x (M, K) bf16 -> (codes (M, K/2) uint8, E8M0 scales (M, K/32) uint8): the
+    fused grouped-Hadamard + MXFP4 step (also the offline weight quantizer)."""
+    if x.dim() != 2:
+        raise ValueError("x must be (M, K)")
+    M, K = x.shape
+    _need(x, "x", torch.bfloat16, (M, K))
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((M, K // 32), dtype=torch.uint8, device=x.device)
+    svdq_mxfp4_quantize(x.data_ptr(), M, K, hadamard_group, codes.data_ptr(), scales.data_ptr(), stream)
+    return codes, scales
+
+
+class MXFP4Linear:
+    """The FP-Quant MXFP4 linear on the current CUDA device: y = alpha * Q(x R^T) Q(W')^T
+    with qweight (N, K/2) and wscales (N, K/32) E8M0 bytes of the rotated weight."""
+
+    def __init__(self, qweight, wscales, alpha: float = 1.0, hadamard_group: int = 32, stream=None):
+        N, K2 = qweight.shape
+        K = 2 * K2
+        _need(qweight, "qweight", qweight.dtype, (N, K // 2))
+        _need(wscales, "wscales", wscales.dtype, (N, K // 32))
+        if qweight.dtype not in (torch.int8, torch.uint8) or wscales.dtype != torch.uint8:
+            raise TypeError("qweight int8/uint8, wscales uint8 (E8M0 bytes)")
+        self.K, self.N, self.group = K, N, hadamard_group
+        d = svdq_mxfp4_desc(K=K, N=N, hadamard_group=hadamard_group, qweight=qweight.data_ptr(),
+                            wscales=wscales.data_ptr(), alpha=float(alpha))
+        self.handle = svdq_mxfp4_create(d, stream)
+        self._ws = None
+
+    def workspace(self, M: int) -> torch.Tensor:
+        nbytes = svdq_mxfp4_workspace_bytes(self.handle, M)
+        if self._ws is None or self._ws.numel() < nbytes:
+            self._ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device="cuda")
+        return self._ws
+
+    def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        M = x.shape[0]
+        _need(x, "x", torch.bfloat16, (M, self.K))
+        y = torch.empty((M, self.N), dtype=torch.bfloat16, device=x.device) if out is None else out
+        _need(y, "y", torch.bfloat16, (M, self.N))
+        svdq_mxfp4_forward(self.handle, x.data_ptr(), M, y.data_ptr(), self.workspace(M).data_ptr(), stream)
+        return y
+
+    __call__ = forward
+
+    def device_status(self) -> int:
+        return svdq_mxfp4_device_status(self.handle)
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            svdq_mxfp4_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def svdq_device_status(handle) -> int:

@@ -40,6 +40,12 @@
 // Every wait is bounded; on expiry the CTA records an error and skips its
 // remaining work.  Both CTAs always reach the final cluster barrier, so
 // neither exits while the other may still touch its shared memory.
+//
+// The MX instantiation serves the MXFP4 matmul of "Rotate in quantization and
+// its vLLM implementation", section 3.3 (FP-Quant): E2M1 operands with one
+// UE8M0 (power-of-two) scale per 32 K elements, stored in the same 512-byte
+// atoms with the two block scales of each 64-element K step in bytes j = 0, 1
+// (bytes 2, 3 zero), and no rank-R branch (R = 0): y = bf16(alpha * acc).
 #include <cuda_runtime.h>
 
 #include <map>
@@ -103,7 +109,7 @@ __device__ __forceinline__ uint64_t sdesc_rows(uint32_t saddr, int row_bytes) {
          ((uint64_t)((8u * (uint32_t)row_bytes) >> 4) << 32) | (1ull << 46) | (layout << 61);
 }
 
-template <int kStages>
+template <int kStages, bool MX>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                            const __grid_constant__ CUtensorMap tm_l, const __grid_constant__ CUtensorMap tm_pu,
@@ -203,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       p.sfb + ((size_t)(2 * nt + h) * p.ka_pad + (size_t)kt * kAtoms) * kSfAtomBytes, kSfbBytes / 2,
                       sb);
           issued = g + 1;
-          if (kt == p.k_tiles - 1) {
+          if (kt == p.k_tiles - 1 && p.R > 0) {
             // This CTA's L rows and proj_up' half, read after the K loop.
             if (it >= 1 && !wait_bounded(smem_u32(lr_free), (it - 1) & 1, abort_flag, p.err, kErrGemmTimeout)) {
               stop = true;
@@ -224,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0 && leader) {
-      const uint32_t idesc_main = idesc_nvfp4(BM, BN);
+      const uint32_t idesc_main = MX ? idesc_mxfp4(BM, BN) : idesc_nvfp4(BM, BN);
       const uint32_t idesc_lr = idesc_bf16_f32(BM, BN);
       int g = 0, it = 0;
       bool ok = true;
@@ -246,26 +252,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t st = smem_u32(stages + s * kStageBytes);
           const uint32_t sf = tmem + kColSf + (uint32_t)b * kSfCols;
 #pragma unroll
-          for (int kb = 0; kb < kAtoms; ++kb)
-            mma_nvfp4_pair(tmem + kColAcc, sdesc_rows(st + kb * 32, kKTileBytes),
-                           sdesc_rows(st + kABytes + kb * 32, kKTileBytes), idesc_main, sf + 4 * kb,
-                           sf + 16 + 8 * kb, (kt | kb) != 0);
+          for (int kb = 0; kb < kAtoms; ++kb) {
+            if (MX)
+              mma_mxfp4_pair(tmem + kColAcc, sdesc_rows(st + kb * 32, kKTileBytes),
+                             sdesc_rows(st + kABytes + kb * 32, kKTileBytes), idesc_main, sf + 4 * kb,
+                             sf + 16 + 8 * kb, (kt | kb) != 0);
+            else
+              mma_nvfp4_pair(tmem + kColAcc, sdesc_rows(st + kb * 32, kKTileBytes),
+                             sdesc_rows(st + kABytes + kb * 32, kKTileBytes), idesc_main, sf + 4 * kb,
+                             sf + 16 + 8 * kb, (kt | kb) != 0);
+          }
           tc_commit_pair(smem_u32(&empty[s]), kPairMask);
         }
         if (!ok) break;
-        if (!wait_bounded(smem_u32(lr_full), it & 1, abort_flag, p.err, kErrGemmTimeout)) {
-          ok = false;
-          break;
+        if (p.R > 0) {                                       // no rank-R branch when R == 0
+          if (!wait_bounded(smem_u32(lr_full), it & 1, abort_flag, p.err, kErrGemmTimeout)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t la = smem_u32(LRB), pa = la + lr_half_bytes;
+          const int per_box = p.lr_row_bytes / 32;           // K = 16 bf16 = 32 bytes per MMA
+          for (int kk = 0; kk < p.R / 16; ++kk) {
+            const int off = (kk / per_box) * lr_box_bytes + (kk % per_box) * 32;
+            mma_bf16_pair(tmem + kColAcc, sdesc_rows(la + off, p.lr_row_bytes),
+                          sdesc_rows(pa + off, p.lr_row_bytes), idesc_lr, 1u);
+          }
+          tc_commit_pair(smem_u32(lr_free), kPairMask);
         }
-        tc_fence_after_sync();
-        const uint32_t la = smem_u32(LRB), pa = la + lr_half_bytes;
-        const int per_box = p.lr_row_bytes / 32;           // K = 16 bf16 = 32 bytes per MMA
-        for (int kk = 0; kk < p.R / 16; ++kk) {
-          const int off = (kk / per_box) * lr_box_bytes + (kk % per_box) * 32;
-          mma_bf16_pair(tmem + kColAcc, sdesc_rows(la + off, p.lr_row_bytes), sdesc_rows(pa + off, p.lr_row_bytes),
-                        idesc_lr, 1u);
-        }
-        tc_commit_pair(smem_u32(lr_free), kPairMask);
         tc_commit_pair(smem_u32(acc_full), kPairMask);
       }
     }
@@ -472,7 +486,7 @@ int max_active_pairs(size_t smem) {
   auto f = cache.find(key);
   if (f != cache.end()) return f->second;
   int n = 0;
-  if (ensure_smem_limit(gemm_nvfp4_pair_kernel<kStages>, smem) == cudaSuccess) {
+  if (ensure_smem_limit(gemm_nvfp4_pair_kernel<kStages, false>, smem) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -484,7 +498,7 @@ int max_active_pairs(size_t smem) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel<kStages>, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel<kStages, false>, &cfg) != cudaSuccess) n = 0;
   }
   cudaGetLastError();   // clear a failed query
   cache[key] = n;
@@ -496,9 +510,9 @@ int max_active_pairs_for(int R) {
   return pair_stages(R) == kMaxStages ? max_active_pairs<kMaxStages>(smem) : max_active_pairs<kMaxStages - 1>(smem);
 }
 
-template <int kStages>
+template <int kStages, bool MX>
 cudaError_t launch_pair(const GemmLaunch& L, const PParams& p, size_t smem, int max_pairs, cudaStream_t stream) {
-  cudaError_t e = ensure_smem_limit(gemm_nvfp4_pair_kernel<kStages>, smem);
+  cudaError_t e = ensure_smem_limit(gemm_nvfp4_pair_kernel<kStages, MX>, smem);
   if (e != cudaSuccess) return e;
   const int tiles = p.m_tiles * p.n_tiles;
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
@@ -516,7 +530,7 @@ cudaError_t launch_pair(const GemmLaunch& L, const PParams& p, size_t smem, int 
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_pair_kernel<kStages>, L.tm_a, L.tm_b, L.tm_l, L.tm_pu, L.tm_y, p);
+  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_pair_kernel<kStages, MX>, L.tm_a, L.tm_b, L.tm_l, L.tm_pu, L.tm_y, p);
 }
 
 }  // namespace
@@ -529,7 +543,7 @@ bool gemm_pair_available(int R) {
 
 cudaError_t launch_gemm_nvfp4_pair(const GemmLaunch& L, cudaStream_t stream) {
   if (L.M <= 0) return cudaSuccess;
-  if (L.R > 128) return cudaErrorInvalidValue;
+  if (L.R > 128 || L.R < 0) return cudaErrorInvalidValue;
   const int stages = pair_stages(L.R);
   const size_t smem = pair_smem_bytes(L.R, stages);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
@@ -552,8 +566,11 @@ cudaError_t launch_gemm_nvfp4_pair(const GemmLaunch& L, cudaStream_t stream) {
   p.lr_row_bytes = gemm_pair_lr_row_bytes(L.R);
   p.lr_boxes = pair_lr_boxes(L.R);
   p.y_mode = (L.N % 8) == 0 ? 3 : 0;
-  return stages == kMaxStages ? launch_pair<kMaxStages>(L, p, smem, max_pairs, stream)
-                              : launch_pair<kMaxStages - 1>(L, p, smem, max_pairs, stream);
+  if (L.mx)
+    return stages == kMaxStages ? launch_pair<kMaxStages, true>(L, p, smem, max_pairs, stream)
+                                : launch_pair<kMaxStages - 1, true>(L, p, smem, max_pairs, stream);
+  return stages == kMaxStages ? launch_pair<kMaxStages, false>(L, p, smem, max_pairs, stream)
+                              : launch_pair<kMaxStages - 1, false>(L, p, smem, max_pairs, stream);
 }
 
 }  // namespace svdq

@@ -311,6 +311,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t m, uint32_t n) {
 __host__ __device__ constexpr uint32_t idesc_nvfp4(uint32_t m, uint32_t n) {
   return (1u << 7) | (1u << 10) | ((n >> 3) << 17) | (0u << 23) | ((m >> 4) << 24);
 }
+// The same with UE8M0 scales (bit 23: scale format), for MXFP4 (block 32);
+// scale data ids 0, so the MMA reads bytes 0-1 of each scale column.
+__host__ __device__ constexpr uint32_t idesc_mxfp4(uint32_t m, uint32_t n) {
+  return (1u << 7) | (1u << 10) | ((n >> 3) << 17) | (1u << 23) | ((m >> 4) << 24);
+}
 
 // --------------------------------------------------------------------------
 // CTA pairs (tcgen05 .cta_group::2): one MMA spans the tensor cores of two
@@ -356,6 +361,18 @@ __device__ __forceinline__ void mma_nvfp4_pair(uint32_t d, uint64_t adesc, uint6
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+// The same pair MMA for MXFP4: one UE8M0 (power-of-two) scale per 32 K
+// elements, two per K = 64 step, read from bytes 0-1 of each scale column.
+__device__ __forceinline__ void mma_mxfp4_pair(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], "
       "p;\n\t}" ::"r"(d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
       : "memory");

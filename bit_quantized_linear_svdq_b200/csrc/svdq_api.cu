@@ -826,3 +826,238 @@ svdq_status svdq_device_status(const svdq_linear* h, int* flags) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- MXFP4 with a grouped Hadamard (FP-Quant)
+
+struct svdq_mxfp4 {
+  int device;
+  int K, N, Kp, k_tiles, ka_pad, group;
+  float alpha;
+  uint8_t* qw;            // (N, Kp/2) packed E2M1, rows zero-padded to Kp
+  uint8_t* sfb;           // weight E8M0 scale atoms ((ceil(N/128) rounded up to even) x ka_pad x 512 B)
+  float* alpha_v;         // (roundup(N, 256)) alpha for every column
+  unsigned* err;          // [0] device error word, [1] create-time checks
+  CUtensorMap tm_b;       // qw: box {128, 128}, 128B swizzle
+};
+
+namespace {
+
+// (N, K/32) row-major E8M0 bytes -> the GEMM's atoms: the two block scales of
+// each 64-element K step in bytes 0, 1 of the row's 32-bit atom word (bytes 2,
+// 3 and every atom past K stay zero from the memset).  bad bit 1: a NaN byte.
+__global__ void repack_mx_scales(const uint8_t* __restrict__ ws, uint8_t* __restrict__ sfb, int N, int G, int ka_pad,
+                                 unsigned* bad) {
+  const long long total = (long long)N * G;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
+    const int n = (int)(i / G), g = (int)(i % G);
+    const uint8_t b = ws[i];
+    if (b == 0xFF) atomicOr(bad, 1u);
+    sfb[((size_t)(n >> 7) * ka_pad + (g >> 1)) * svdq::kSfAtomBytes + svdq::sf_atom_offset(n & 127, g & 1)] = b;
+  }
+}
+
+__global__ void fill_f32(float* p, float v, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = v;
+}
+
+void free_mx(svdq_mxfp4* h) {
+  if (!h) return;
+  cudaFree(h->qw);
+  cudaFree(h->sfb);
+  cudaFree(h->alpha_v);
+  cudaFree(h->err);
+  delete h;
+}
+
+struct MxWs {
+  size_t codes, sfa, total;
+};
+MxWs mx_ws_layout(const svdq_mxfp4* h, int M) {
+  MxWs w;
+  w.codes = 0;
+  w.sfa = align256((size_t)M * (h->Kp / 2));
+  w.total = align256(w.sfa + (size_t)((M + 127) / 128) * h->ka_pad * svdq::kSfAtomBytes);
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+svdq_status svdq_mxfp4_create(svdq_mxfp4** out, const svdq_mxfp4_desc* d, void* stream_) {
+  if (!out) return SVDQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!d || !d->qweight || !d->wscales) return SVDQ_ERR_INVALID_ARG;
+  if (d->K <= 0 || d->N <= 0 || d->K % 32 != 0) return SVDQ_ERR_SHAPE;
+  if (d->hadamard_group != 0 && d->hadamard_group != 32) return SVDQ_ERR_SHAPE;
+  if ((long long)d->K * d->N > (1LL << 40)) return SVDQ_ERR_SHAPE;
+  if (!std::isfinite(d->alpha)) return SVDQ_ERR_INVALID_ARG;
+  int dev = 0, major = 0, minor = 0;
+  SVDQ_CUDA(cudaGetDevice(&dev));
+  SVDQ_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  SVDQ_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+  if (major != 10 || minor != 0) {
+    g_last_error = "requires an sm_100 (B200) device";
+    return SVDQ_ERR_UNSUPPORTED;
+  }
+  if (!svdq::gemm_pair_available(0)) {
+    g_last_error = "the pair GEMM does not fit on this device";
+    return SVDQ_ERR_UNSUPPORTED;
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  svdq_mxfp4* h = new svdq_mxfp4();
+  std::memset(h, 0, sizeof(*h));
+  h->device = dev;
+  h->K = d->K;
+  h->N = d->N;
+  h->group = d->hadamard_group;
+  h->alpha = d->alpha;
+  h->Kp = (d->K + 127) / 128 * 128;
+  h->k_tiles = (h->Kp + 255) / 256;
+  h->ka_pad = 4 * h->k_tiles;
+  const int n_tiles_even = (((d->N + 127) / 128) + 1) & ~1;
+  const int Npad256 = (d->N + 255) / 256 * 256;
+  cudaError_t e;
+  auto fail = [&](svdq_status st) {
+    free_mx(h);
+    return st;
+  };
+#define MX_CUDA(call)                             \
+  do {                                            \
+    e = (call);                                   \
+    if (e != cudaSuccess) {                       \
+      cuda_fail(e, #call);                        \
+      return fail(SVDQ_ERR_CUDA);                 \
+    }                                             \
+  } while (0)
+  MX_CUDA(cudaMalloc(&h->qw, (size_t)d->N * (h->Kp / 2)));
+  MX_CUDA(cudaMalloc(&h->sfb, (size_t)n_tiles_even * h->ka_pad * svdq::kSfAtomBytes));
+  MX_CUDA(cudaMalloc(&h->alpha_v, (size_t)Npad256 * sizeof(float)));
+  MX_CUDA(cudaMalloc(&h->err, 2 * sizeof(unsigned)));
+  MX_CUDA(cudaMemsetAsync(h->err, 0, 2 * sizeof(unsigned), stream));
+  MX_CUDA(cudaMemset2DAsync(h->qw, h->Kp / 2, 0, h->Kp / 2, d->N, stream));
+  MX_CUDA(cudaMemcpy2DAsync(h->qw, h->Kp / 2, d->qweight, d->K / 2, d->K / 2, d->N, cudaMemcpyDeviceToDevice, stream));
+  MX_CUDA(cudaMemsetAsync(h->sfb, 0, (size_t)n_tiles_even * h->ka_pad * svdq::kSfAtomBytes, stream));
+  repack_mx_scales<<<grid_for((long long)d->N * (d->K / 32)), 256, 0, stream>>>(
+      static_cast<const uint8_t*>(d->wscales), h->sfb, d->N, d->K / 32, h->ka_pad, h->err + 1);
+  MX_CUDA(cudaGetLastError());
+  fill_f32<<<grid_for(Npad256), 256, 0, stream>>>(h->alpha_v, d->alpha, Npad256);
+  MX_CUDA(cudaGetLastError());
+  unsigned bad = 0;
+  MX_CUDA(cudaMemcpyAsync(&bad, h->err + 1, sizeof(unsigned), cudaMemcpyDeviceToHost, stream));
+  MX_CUDA(cudaStreamSynchronize(stream));
+#undef MX_CUDA
+  if (bad & 1u) {
+    g_last_error = "wscales holds an E8M0 NaN (0xFF)";
+    return fail(SVDQ_ERR_INVALID_ARG);
+  }
+  svdq_status s;
+  if ((s = make_tmap(&h->tm_b, h->qw, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->Kp / 2, d->N, h->Kp / 2, 128, 128)) != SVDQ_OK)
+    return fail(s);
+  *out = h;
+  return SVDQ_OK;
+}
+
+void svdq_mxfp4_destroy(svdq_mxfp4* h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  free_mx(h);
+}
+
+size_t svdq_mxfp4_workspace_bytes(const svdq_mxfp4* h, int M) {
+  if (!h || M <= 0) return 0;
+  return mx_ws_layout(h, M).total;
+}
+
+svdq_status svdq_mxfp4_quantize(const void* x, int M, int K, int hadamard_group, void* codes, void* scales,
+                                void* stream) {
+  if (M < 0 || K <= 0 || K % 32 != 0) return M < 0 ? SVDQ_ERR_INVALID_ARG : SVDQ_ERR_SHAPE;
+  if (hadamard_group != 0 && hadamard_group != 32) return SVDQ_ERR_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  if (!x || !codes || !scales || !aligned16(x) || !aligned16(codes)) return SVDQ_ERR_INVALID_ARG;
+  svdq::MxQuantLaunch q;
+  q.x = x;
+  q.codes = static_cast<uint8_t*>(codes);
+  q.scales = static_cast<uint8_t*>(scales);
+  q.M = M;
+  q.K = K;
+  q.Kp = K;
+  q.codes_pitch = K / 2;
+  q.scales_pitch = K / 32;
+  q.ka_pad = 0;
+  q.group = hadamard_group;
+  q.tiled = false;
+  cudaError_t e = svdq::launch_quantize_mx(q, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "quantize_mx launch");
+  return SVDQ_OK;
+}
+
+svdq_status svdq_mxfp4_forward(const svdq_mxfp4* h, const void* x, int M, void* y, void* workspace, void* stream_) {
+  if (!h || M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!x || !y || !aligned16(x) || !aligned16(y)) return SVDQ_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SVDQ_ERR_WORKSPACE;
+  int dev = -1;
+  SVDQ_CUDA(cudaGetDevice(&dev));
+  if (dev != h->device) {
+    g_last_error = "current device differs from the device the handle was created on";
+    return SVDQ_ERR_INVALID_ARG;
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  const MxWs w = mx_ws_layout(h, M);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  svdq::MxQuantLaunch q;
+  q.x = x;
+  q.codes = ws + w.codes;
+  q.scales = ws + w.sfa;
+  q.M = M;
+  q.K = h->K;
+  q.Kp = h->Kp;
+  q.codes_pitch = h->Kp / 2;
+  q.scales_pitch = 0;
+  q.ka_pad = h->ka_pad;
+  q.group = h->group;
+  q.tiled = true;
+  cudaError_t e = svdq::launch_quantize_mx(q, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "quantize_mx launch");
+  svdq::GemmLaunch g;
+  std::memset(&g, 0, sizeof(g));
+  svdq_status s;
+  if ((s = make_tmap(&g.tm_a, ws + w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->Kp / 2, M, h->Kp / 2, 128, 128)) !=
+      SVDQ_OK)
+    return s;
+  g.tm_b = h->tm_b;
+  g.tm_l = h->tm_b;      // no rank-R branch: the L and proj_up maps are never read
+  g.tm_pu = h->tm_b;
+  if (h->N % 8 == 0 &&
+      (s = make_tmap(&g.tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->N, M, (uint64_t)h->N * 2, 64, 32)) != SVDQ_OK)
+    return s;
+  else if (h->N % 8 != 0)
+    g.tm_y = h->tm_b;
+  g.sfa = ws + w.sfa;
+  g.sfb = h->sfb;
+  g.alpha = h->alpha_v;
+  g.y = y;
+  g.err = h->err;
+  g.M = M;
+  g.N = h->N;
+  g.R = 0;
+  g.k_tiles = h->k_tiles;
+  g.ka_pad = h->ka_pad;
+  g.mx = true;
+  e = svdq::launch_gemm_nvfp4_pair(g, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "mxfp4 gemm launch");
+  return SVDQ_OK;
+}
+
+svdq_status svdq_mxfp4_device_status(const svdq_mxfp4* h, int* flags) {
+  if (!h) return SVDQ_ERR_INVALID_ARG;
+  unsigned v = 0;
+  SVDQ_CUDA(cudaDeviceSynchronize());
+  SVDQ_CUDA(cudaMemcpy(&v, h->err, sizeof(unsigned), cudaMemcpyDeviceToHost));
+  SVDQ_CUDA(cudaMemset(h->err, 0, sizeof(unsigned)));
+  if (flags) *flags = (int)v;
+  return v ? SVDQ_ERR_DEVICE : SVDQ_OK;
+}
+
+}  // extern "C"

@@ -32,6 +32,22 @@ struct QuantLaunch {
 };
 cudaError_t launch_quantize_act(const QuantLaunch& p, cudaStream_t stream);
 
+// Grouped-Hadamard + MXFP4 quantizer (FP-Quant forward): x bf16 (M, K), K a
+// multiple of 32 -> codes (row pitch codes_pitch) and E8M0 scales, either
+// row-major (M, K/32) or in the GEMM's 512-byte atoms (two block scales per
+// 64-element K step in bytes 0-1, bytes 2-3 zero), with codes and atoms zero
+// up to Kp and ka_pad.  group: 0 (no rotation) or 32.
+struct MxQuantLaunch {
+  const void* x;
+  uint8_t* codes;
+  uint8_t* scales;
+  int M, K, Kp;             // Kp: codes and atoms written up to Kp (tiled) or K (row-major)
+  int codes_pitch, scales_pitch, ka_pad;
+  int group;
+  bool tiled;
+};
+cudaError_t launch_quantize_mx(const MxQuantLaunch& p, cudaStream_t stream);
+
 // Standalone Walsh-Hadamard transform of rows of length 2^log2n (<= 2^15),
 // in place; dtype 0 = bf16, 1 = fp16.
 cudaError_t launch_hadamard_transform(void* x, int rows, int log2n, int dtype, cudaStream_t stream);
@@ -57,6 +73,7 @@ struct GemmLaunch {
   int M, N, R;
   int k_tiles;              // Kp rounded up to 256, divided by 256
   int ka_pad;               // K atoms per 128-row scale tile (= 4 * k_tiles)
+  bool mx;                  // pair kernel only: MXFP4 operands (UE8M0 scale per 32, bytes 0-1 of each atom word)
 };
 cudaError_t launch_gemm_nvfp4_lr(const GemmLaunch& p, cudaStream_t stream);
 

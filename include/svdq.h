@@ -250,6 +250,78 @@ SVDQ_API svdq_status svdq_quantize_weight(const void* w, int N, int K, int rotat
  */
 SVDQ_API svdq_status svdq_device_status(const svdq_linear* h, int* flags);
 
+/*
+ * ---------------------------------------------------------------------------
+ * MXFP4 with a grouped Hadamard rotation: the FP-Quant forward of "Rotate in
+ * quantization and its vLLM implementation", section 3.3 (FPQuantConfig with
+ * hadamard_group_size 32, forward_dtype "mxfp4", forward_method "abs_max";
+ * the fused rotate-and-quantize step followed by the MXFP4 matmul to bf16):
+ *
+ *   x_hat = x R^T        R = blockdiag(H_32 / sqrt(32)) (or the identity, group 0)
+ *   y     = bf16( alpha * Q(x_hat) Q(W')^T )      W' = W R^T, quantized offline
+ *
+ * Q() is MXFP4: E2M1 codes, two per byte (element 2j in the low nibble of byte
+ * j), one E8M0 scale byte per 32 consecutive K elements (value 2^(byte - 127),
+ * 255 = NaN).  The page names the method "abs_max" without its formula; this
+ * library takes, for each block, the smallest power of two s with
+ * amax(|x_hat|) / s <= 6 (the largest E2M1 magnitude), exponent clamped to
+ * [-127, 127] (a zero block gets byte 0, a block holding NaN byte 255 and zero
+ * codes), and code = e2m1_rne_satfinite(x_hat / s).  Rotation arithmetic is
+ * fp32: butterfly stages h = 1, 2, 4, 8, 16, then one multiply by
+ * fp32(1/sqrt(32)).  There is no smoothing and no rank-R branch.
+ * ---------------------------------------------------------------------------
+ */
+typedef struct svdq_mxfp4 svdq_mxfp4;
+
+typedef struct {
+  int K;                      /* input features, a positive multiple of 32 */
+  int N;                      /* output features, >= 1 */
+  int hadamard_group;         /* 32: the rotation above; 0: none */
+  const void* qweight;        /* (N, K/2)  uint8: packed E2M1 of the rotated weight W' (device) */
+  const void* wscales;        /* (N, K/32) uint8: E8M0 scale bytes of W', row-major (device); 255 is refused */
+  float alpha;                /* the matmul's output scale (finite) */
+} svdq_mxfp4_desc;
+
+/*
+ * svdq_mxfp4_create -- copy the weight codes (rows padded for TMA) and re-tile
+ * the weight scales into the tensor-core scale layout in library-owned device
+ * memory; synchronizes `stream`, after which the sources may be freed.
+ * SVDQ_ERR_SHAPE for K % 32 != 0 or a group other than 0 / 32;
+ * SVDQ_ERR_INVALID_ARG for a NaN scale byte or a non-finite alpha.
+ */
+SVDQ_API svdq_status svdq_mxfp4_create(svdq_mxfp4** out, const svdq_mxfp4_desc* desc, void* stream);
+
+/* Free the handle and its device memory.  NULL is a no-op.  Synchronizes the device. */
+SVDQ_API void svdq_mxfp4_destroy(svdq_mxfp4* h);
+
+/* Bytes of device workspace svdq_mxfp4_forward needs for M rows (0 for M == 0). */
+SVDQ_API size_t svdq_mxfp4_workspace_bytes(const svdq_mxfp4* h, int M);
+
+/*
+ * svdq_mxfp4_quantize -- the fused rotate-and-quantize step alone, in the
+ * public layout (no handle; also the offline weight quantizer: pass W's rows).
+ *   x       (M, K)    bf16 in, 16-byte aligned; K a positive multiple of 32
+ *   codes   (M, K/2)  uint8 out: packed E2M1, element 2j in the low nibble; 16-byte aligned
+ *   scales  (M, K/32) uint8 out: E8M0 bytes, row-major
+ *   hadamard_group    32 or 0
+ * M == 0 is a no-op.  Caller-owned device buffers; asynchronous on `stream`.
+ */
+SVDQ_API svdq_status svdq_mxfp4_quantize(const void* x, int M, int K, int hadamard_group, void* codes, void* scales,
+                                         void* stream);
+
+/*
+ * svdq_mxfp4_forward -- y (M, N) bf16 = alpha * Q(x R^T) Q(W')^T: the fused
+ * rotate-and-quantize kernel writes codes and scale tiles into `workspace`,
+ * then the block-scaled MXFP4 GEMM (tcgen05, 256 x 256 tiles on CTA pairs)
+ * writes y.  x 16-byte aligned; workspace >= svdq_mxfp4_workspace_bytes(h, M)
+ * bytes, 256-byte aligned, caller-owned, not shared by concurrent calls.
+ */
+SVDQ_API svdq_status svdq_mxfp4_forward(const svdq_mxfp4* h, const void* x, int M, void* y, void* workspace,
+                                        void* stream);
+
+/* As svdq_device_status, for an MXFP4 handle (bit 1: the GEMM's bounded wait expired). */
+SVDQ_API svdq_status svdq_mxfp4_device_status(const svdq_mxfp4* h, int* flags);
+
 /* Static text for a status code. */
 SVDQ_API const char* svdq_status_string(svdq_status s);
 

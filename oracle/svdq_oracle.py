@@ -359,3 +359,103 @@ def int_absmax_quantize(x, bits: int, signed: bool = True):
     scale = np.max(np.abs(x)) / qmax
     q = np.clip(np.rint(x / scale), qmin, qmax).astype(np.int64)
     return scale, q, q * scale
+
+
+# ----------------------------------------------------------------------------
+# MXFP4 with a grouped Hadamard: the FP-Quant forward ("Rotate in quantization
+# and its vLLM implementation", section 3.3).  The page gives the configuration
+# (hadamard_group_size = 32, forward_dtype "mxfp4", forward_method "abs_max"),
+# the fused rotate-and-quantize step and the matmul y = alpha * (x_q w_q^T) in
+# bf16.  Readings, where the page is silent:
+#   * MXFP4 = E2M1 codes (the grid above) in blocks of 32 consecutive K
+#     elements, each block with one shared power-of-two scale stored as an
+#     E8M0 byte (value 2^(byte - 127), byte 255 = NaN), the OCP MX format;
+#   * "abs_max": the block scale is the smallest power of two s with
+#     amax / s <= 6 (the largest E2M1 magnitude), i.e. s = 2^ceil(log2(amax / 6)),
+#     so the block's largest magnitude lands inside the grid (the absmax rule of
+#     the page's section 1 under a power-of-two constraint); the exponent is
+#     clamped to [-127, 127]; a zero block gets 2^-127 (byte 0) and a NaN block
+#     byte 255 with zero codes;
+#   * code = e2m1_rne_satfinite(x_hat / s) (exact: s is a power of two);
+#   * the rotation is the fp32 butterfly of the 128-block case with block 32
+#     (x_hat = fp32(butterfly_32(x) * fp32(1/sqrt(32)))), applied to the
+#     activations online and to the weight rows offline (W' = W R^T, rows
+#     rotated like activation rows); no smoothing and no rank-R branch;
+#   * weight scales are stored like the activation scales: (N, K/32) E8M0
+#     bytes, row-major; alpha is one fp32 scalar.
+# ----------------------------------------------------------------------------
+
+def e8m0_decode(bits: np.ndarray) -> np.ndarray:
+    """E8M0 byte -> float64 value 2^(byte - 127); byte 255 is NaN."""
+    b = np.asarray(bits, dtype=np.uint8).astype(np.int64)
+    return np.where(b == 255, np.nan, np.exp2(b - 127.0))
+
+
+def mx_abs_max_exponent(amax: np.ndarray) -> np.ndarray:
+    """Smallest integer e with 2^e >= amax / 6 (amax > 0 finite), clamped to
+    [-127, 127]; -127 for amax == 0.  Decided on exact values: float64 holds
+    every fp32 amax and every 6 * 2^e exactly."""
+    a = np.asarray(amax, dtype=np.float64)
+    e = np.full(a.shape, -127, dtype=np.int64)
+    pos = a > 0
+    # frexp: a = f * 2^k, f in [0.5, 1); a / 6 = (f / 6) * 2^k; start from a
+    # close guess and correct it with exact comparisons against 6 * 2^e.
+    f, k = np.frexp(np.where(pos, a, 1.0))
+    guess = k.astype(np.int64) - 2
+    for _ in range(3):
+        too_small = 6.0 * np.exp2(guess.astype(np.float64)) < a          # 2^guess < a / 6
+        guess = np.where(too_small, guess + 1, guess)
+        too_big = 6.0 * np.exp2(guess.astype(np.float64) - 1.0) >= a     # 2^(guess-1) >= a / 6
+        guess = np.where(too_big, guess - 1, guess)
+    e = np.where(pos, guess, e)
+    return np.clip(e, -127, 127)
+
+
+def quantize_mxfp4_rows(v32: np.ndarray):
+    """MXFP4 quantization of fp32 rows: one E8M0 scale per 32 consecutive
+    elements (the abs_max reading above).  Returns (packed codes (rows, K/2)
+    uint8, scale bytes (rows, K/32) uint8)."""
+    v32 = np.asarray(v32, dtype=np.float32)
+    rows, K = v32.shape
+    blk = v32.reshape(rows, K // 32, 32).astype(np.float64)
+    amax = np.max(np.abs(blk), axis=2)
+    nan_blk = np.isnan(amax)
+    e = mx_abs_max_exponent(np.where(nan_blk, 0.0, np.minimum(amax, np.finfo(np.float64).max)))
+    s = np.exp2(e.astype(np.float64))
+    with np.errstate(over="ignore", invalid="ignore"):
+        q = blk / s[:, :, None]                                       # exact: power-of-two scale
+    codes = e2m1_encode_rne_satfinite(q)
+    codes = np.where(nan_blk[:, :, None], np.uint8(0), codes).astype(np.uint8)
+    sbytes = np.where(nan_blk, 255, e + 127).astype(np.uint8)
+    return pack_e2m1(codes.reshape(rows, K)), sbytes
+
+
+def dequantize_mxfp4(codes: np.ndarray, scale_bytes: np.ndarray) -> np.ndarray:
+    """Packed codes (rows, K/2) + E8M0 bytes (rows, K/32) -> float64 (rows, K)."""
+    c = e2m1_decode(unpack_e2m1(codes))
+    return c * np.repeat(e8m0_decode(scale_bytes), 32, axis=1)
+
+
+def fpquant_quantize(x_bits: np.ndarray, group: int = 32):
+    """The fused rotate-and-quantize step: x (bf16 bits, (M, K)) -> x_hat =
+    blockwise rotation by H_group / sqrt(group) in fp32 (group 0: none) ->
+    MXFP4 (codes (M, K/2), scale bytes (M, K/32), x_hat fp32)."""
+    xh = bf16_to_f32(x_bits).astype(np.float32)
+    if group:
+        xh = rotate_rows_fp32(xh, group)
+    codes, scales = quantize_mxfp4_rows(xh)
+    return codes, scales, xh
+
+
+def fpquant_quantize_weight(dense_bits: np.ndarray, group: int = 32):
+    """Offline weight step: dense bf16 W (N, K) -> rows rotated like activation
+    rows -> MXFP4 (qweight (N, K/2), wscales (N, K/32))."""
+    codes, scales, _ = fpquant_quantize(dense_bits, group)
+    return codes, scales
+
+
+def fpquant_forward(x_bits, qweight, wscales, alpha: float, group: int = 32, rows=None) -> np.ndarray:
+    """y (M, N) float64 = alpha * (Q(x_hat) Q(W')^T), Q = MXFP4 dequantization."""
+    xb = x_bits if rows is None else x_bits[rows]
+    codes, scales, _ = fpquant_quantize(xb, group)
+    return np.float64(alpha) * (dequantize_mxfp4(codes, scales) @ dequantize_mxfp4(qweight, wscales).T)

@@ -22,7 +22,8 @@ def test_exports_every_declared_symbol(lib):
         "svdq_linear_forward", "svdq_linear_forward_host", "svdq_device_status", "svdq_status_string",
         "svdq_last_error", "svdq_version", "svdq_linear_forward_quantize", "svdq_linear_forward_gemm",
         "svdq_linear_forward_noalloc", "svdq_quantize_weight", "svdq_hadamard_transform",
-        "svdq_linear_gemm_kernel"}
+        "svdq_linear_gemm_kernel", "svdq_mxfp4_create", "svdq_mxfp4_destroy", "svdq_mxfp4_workspace_bytes",
+        "svdq_mxfp4_quantize", "svdq_mxfp4_forward", "svdq_mxfp4_device_status"}
     for n in names:
         assert hasattr(lib, n), n
 
@@ -112,3 +113,30 @@ def test_quantize_weight_argument_errors(lib, args, status):
 def test_hadamard_transform_argument_errors(lib, args, status):
     x, rows, n, dt = args
     assert lib.svdq_hadamard_transform(x, rows, n, dt, None) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(K=48), 2),                 # K % 32
+    (dict(K=0), 2),
+    (dict(N=0), 2),
+    (dict(hadamard_group=16), 2),
+    (dict(qweight=None), 1),
+    (dict(wscales=None), 1),
+    (dict(alpha=float("inf")), 1),
+])
+def test_mxfp4_create_rejects_bad_desc_on_host(lib, kw, status):
+    base = dict(K=256, N=256, hadamard_group=32, qweight=1, wscales=1, alpha=1.0)
+    base.update(kw)
+    h = ctypes.c_void_p(123)
+    st = lib.svdq_mxfp4_create(ctypes.byref(h), ctypes.byref(S.svdq_mxfp4_desc(**base)), None)
+    assert st == status and h.value is None
+
+
+def test_mxfp4_quantize_rejects_bad_args_on_host(lib):
+    assert lib.svdq_mxfp4_quantize(16, 4, 48, 32, 16, 16, None) == 2     # K % 32
+    assert lib.svdq_mxfp4_quantize(16, 4, 64, 8, 16, 16, None) == 2      # group
+    assert lib.svdq_mxfp4_quantize(None, 4, 64, 32, 16, 16, None) == 1   # null x
+    assert lib.svdq_mxfp4_quantize(24, 4, 64, 32, 16, 16, None) == 1     # misaligned x
+    assert lib.svdq_mxfp4_quantize(16, 0, 64, 32, 16, 16, None) == 0     # M == 0: no-op
+    assert lib.svdq_mxfp4_workspace_bytes(None, 4) == 0
+    assert lib.svdq_mxfp4_forward(None, 16, 4, 16, 256, None) == 1

@@ -688,3 +688,116 @@ def test_hadamard_transform_involution_and_norm(n, dtype):
     np.testing.assert_allclose(np.linalg.norm(yy, axis=1), np.linalg.norm(x0, axis=1), rtol=4 * eps)
     back = dec(O.hadamard_transform(y, n, dtype)).astype(np.float64)
     assert np.max(np.abs(back - x0)) <= 4 * eps * np.abs(x0).max()
+
+
+# ---------------------------------------------------------------- [rot] section 3.3: MXFP4 with a grouped Hadamard (FP-Quant)
+
+def test_e8m0_decode_matches_torch_all_bytes():
+    b = np.arange(256, dtype=np.uint8)
+    ours = O.e8m0_decode(b)
+    ref = torch.from_numpy(b.copy()).view(torch.float8_e8m0fnu).float().numpy().astype(np.float64)
+    assert np.isnan(ours[255]) and np.isnan(ref[255])
+    np.testing.assert_array_equal(ours[:255][ref[:255] > 0], ref[:255][ref[:255] > 0])
+    assert ours[127] == 1.0 and ours[0] == 2.0 ** -127 and ours[254] == 2.0 ** 127
+
+
+def test_mx_abs_max_exponent_exact_boundaries():
+    # The smallest power of two s with amax / s <= 6, checked by exact rational
+    # arithmetic at every boundary amax = 6 * 2^e and one fp32 ulp either side.
+    def brute(a: Fraction) -> int:
+        e = -200
+        while Fraction(6) * Fraction(2) ** e < a:
+            e += 1
+        return max(-127, min(127, e))
+    checked = 0
+    for e in range(-126, 126):
+        c = np.float32(6.0 * 2.0 ** e)
+        for a in (c, np.nextafter(c, np.float32(np.inf)), np.nextafter(c, np.float32(0))):
+            got = int(O.mx_abs_max_exponent(np.array([float(a)]))[0])
+            assert got == brute(Fraction(float(a))), (e, a, got)
+            checked += 1
+    rng = np.random.default_rng(17)
+    for a in np.exp2(rng.uniform(-140, 128, 300)).astype(np.float32):
+        if not np.isfinite(a) or a == 0:
+            continue
+        assert int(O.mx_abs_max_exponent(np.array([float(a)]))[0]) == brute(Fraction(float(a)))
+        checked += 1
+    assert checked > 900
+    assert O.mx_abs_max_exponent(np.array([0.0]))[0] == -127
+
+
+def test_mxfp4_bruteforce_all_codes_all_scales():
+    # Every E8M0 scale whose 6 * s is a finite fp32 value, all 16 E2M1 codes:
+    # a block holding code * s (with +6s, so amax = 6s) quantizes back to those
+    # codes with scale byte log2(s) + 127.
+    codes = np.arange(16, dtype=np.uint8)
+    vals = O.e2m1_decode(np.concatenate([codes, codes]))            # 32 elements per block
+    blocks, want = [], []
+    for e in range(-127, 126):
+        blocks.append((vals * 2.0 ** e).astype(np.float32))
+        want.append(e + 127)
+    v = np.stack(blocks)
+    assert np.array_equal(v.astype(np.float64), np.stack([vals * 2.0 ** (b - 127) for b in want]))
+    packed, sb = O.quantize_mxfp4_rows(v)
+    np.testing.assert_array_equal(sb[:, 0], want)
+    np.testing.assert_array_equal(O.unpack_e2m1(packed), np.tile(np.concatenate([codes, codes]), (len(want), 1)))
+    np.testing.assert_array_equal(O.dequantize_mxfp4(packed, sb), v.astype(np.float64))
+
+
+def test_mxfp4_ties_zero_nan_inf_blocks():
+    s = 2.0 ** -3
+    row = np.zeros((4, 32), np.float32)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    row[0, :7] = mids * s
+    row[0, 7] = 6 * s
+    row[0, 8:15] = -mids * s
+    row[1, 3] = np.nan
+    row[2, 5] = np.inf
+    row[2, 6] = 1.0
+    # row 3 stays zero
+    packed, sb = O.quantize_mxfp4_rows(row)
+    c = O.unpack_e2m1(packed)
+    np.testing.assert_array_equal(c[0, :7], [0, 2, 2, 4, 4, 6, 6])
+    np.testing.assert_array_equal(c[0, 8:15], np.array([0, 2, 2, 4, 4, 6, 6]) | 8)
+    assert sb[0, 0] == 127 - 3
+    assert sb[1, 0] == 255 and not c[1].any()                       # NaN block: NaN scale, zero codes
+    assert sb[2, 0] == 254 and c[2, 5] == 7 and c[2, 6] == 0         # inf saturates, the rest underflows
+    assert sb[3, 0] == 0 and not c[3].any()                         # zero block: smallest scale
+
+
+@pytest.mark.parametrize("group", [0, 32])
+def test_fpquant_exact_recovery_and_rotation_identity(group):
+    # group 0: activations and weights already on the MXFP4 grid quantize
+    # exactly, so y equals alpha * x W^T in fp64.  group 32: before
+    # quantization the grouped rotation leaves the product unchanged,
+    # (x R^T)(W R^T)^T = x W^T ([rot] 2.1), here through the oracle's fp32
+    # rotation of both operands.
+    rng = np.random.default_rng(61 + group)
+    M, K, N = 3, 128, 5
+
+    def grid(rows):
+        out = np.zeros((rows, K))
+        for r in range(rows):
+            for b in range(K // 32):
+                c = rng.integers(0, 16, 32)
+                c[rng.integers(0, 32)] = 7
+                out[r, 32 * b:32 * (b + 1)] = O.e2m1_decode(c) * 2.0 ** int(rng.integers(-4, 4))
+        return out
+    if group == 0:
+        x, W = grid(M), grid(N)
+        qw, ws = O.fpquant_quantize_weight(_bf16_bits(W), 0)
+        y = O.fpquant_forward(_bf16_bits(x), qw, ws, 0.75, 0)
+        np.testing.assert_array_equal(y, 0.75 * (x @ W.T))
+    else:
+        x = rng.standard_normal((M, K))
+        W = rng.standard_normal((N, K))
+        xb, Wb = _bf16_bits(x), _bf16_bits(W)
+        _, _, xh = O.fpquant_quantize(xb, 32)
+        _, _, wh = O.fpquant_quantize(Wb, 32)
+        ref = O.bf16_to_f32(xb).astype(np.float64) @ O.bf16_to_f32(Wb).astype(np.float64).T
+        got = xh.astype(np.float64) @ wh.astype(np.float64).T
+        assert np.all(np.abs(got - ref) <= 2.0 ** -18 * np.abs(x).sum(1)[:, None] * np.abs(W).max())
+        # the fp32 grouped rotation is the dense H_32 / sqrt(32) up to fp32 rounding
+        H = O.sylvester_hadamard(32) / np.sqrt(32)
+        dense = (O.bf16_to_f32(xb).astype(np.float64).reshape(M, K // 32, 32) @ H.T).reshape(M, K)
+        np.testing.assert_allclose(xh, dense, rtol=0, atol=1e-6 * np.abs(dense).max())
