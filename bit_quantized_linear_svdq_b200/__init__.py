@@ -26,7 +26,7 @@ __all__ = [
     "svdq_last_error", "svdq_version", "svdq_quantize_weight", "quantize_weight", "svdq_hadamard_transform",
     "hadamard_transform", "SVDQLinear", "STATUS", "svdq_mxfp4_desc", "svdq_mxfp4_create", "svdq_mxfp4_destroy",
     "svdq_mxfp4_workspace_bytes", "svdq_mxfp4_quantize", "svdq_mxfp4_forward", "svdq_mxfp4_device_status",
-    "mxfp4_quantize", "MXFP4Linear",
+    "mxfp4_quantize", "MXFP4Linear", "svdq_fp4_mma_loop", "svdq_fp4_mma_loop_status",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -109,6 +109,8 @@ def load_library() -> ctypes.CDLL:
         "svdq_mxfp4_quantize": (ci, [vp, ci, ci, ci, vp, vp, vp]),
         "svdq_mxfp4_forward": (ci, [vp, vp, ci, vp, vp, vp]),
         "svdq_mxfp4_device_status": (ci, [vp, ctypes.POINTER(ci)]),
+        "svdq_fp4_mma_loop": (ci, [ci, ctypes.POINTER(ci), vp]),
+        "svdq_fp4_mma_loop_status": (ci, [ctypes.POINTER(ci)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -327,6 +329,21 @@ class MXFP4Linear:
             self.close()
         except Exception:
             pass
+
+
+def svdq_fp4_mma_loop(iters: int, stream=None) -> int:
+    """Launch the FP4 tensor-rate loop (one CTA per SM); returns the CTA count."""
+    ctas = ctypes.c_int(0)
+    _check(load_library().svdq_fp4_mma_loop(iters, ctypes.byref(ctas), _stream(stream)), "svdq_fp4_mma_loop")
+    return ctas.value
+
+
+def svdq_fp4_mma_loop_status() -> int:
+    flags = ctypes.c_int(0)
+    st = load_library().svdq_fp4_mma_loop_status(ctypes.byref(flags))
+    if st not in (0, 6):
+        raise SvdqError(st, "svdq_fp4_mma_loop_status")
+    return flags.value
 
 
 def svdq_device_status(handle) -> int:

@@ -21,7 +21,7 @@
 // Work decomposition.  A CTA owns 128 token rows and a contiguous slice of
 // K; the K slices of one row tile form a thread-block cluster that reduces
 // its partial L in distributed shared memory (fixed order, deterministic).
-// Inside a CTA (608 threads, one CTA per SM):
+// Inside a CTA (640 threads, one CTA per SM):
 //   warps 0-15      compute: without rotation each thread takes one 16-channel
 //                   block column of two rows (t/8 and t/8 + 64); with rotation
 //                   four threads share a row (32 K elements each).  Smooth
@@ -29,11 +29,16 @@
 //                   store them, in the caller's row-major layout).
 //   warp 16 lane 0  TMA producer: x chunk (128 rows x 128 K, two 128B-swizzled
 //                   boxes), P^T chunk (R x 128) and the smoothing operands into
-//                   a ring of up to 4 stages; the warp owns the TMEM allocation.
+//                   a ring of up to 4 stages; once the compute warps are done
+//                   with a chunk it writes the chunk's staged codes (TMA
+//                   store) and scale atoms (bulk store), and once those and the
+//                   MMAs have read the stage it loads the chunk that reuses it.
+//                   The warp owns the TMEM allocation.
 //   warp 17 lane 0  issues tcgen05.mma (M=128, N=R, K=16, bf16 -> fp32 TMEM)
 //                   for L as soon as a chunk has landed.
-//   warp 18 lane 0  writes a chunk's staged codes (TMA store) and scale atoms
-//                   (bulk store) once the compute warps are done with it.
+//   warps 16-19     once the last MMA has completed (while the compute warps
+//                   finish their last chunks), read the rank-R partial sums of
+//                   TMEM lane quadrants 0-3 and push them to their owner CTA.
 // A stage is reloaded after both the MMAs and the stores have read it.
 //
 // Exact fp32 division without the divide unit.  With y = RZ(1/b) and
@@ -76,9 +81,17 @@ constexpr int kCodeStageBytes = kRows * kChunk / 2;   // 8 KB
 constexpr int kSfStageBytes = 2 * kSfAtomBytes;       // 1 KB
 constexpr int kComputeWarps = 16;
 constexpr int kComputeThreads = 32 * kComputeWarps;
-constexpr int kProducerWarp = kComputeWarps, kMmaWarp = kComputeWarps + 1, kStoreWarp = kComputeWarps + 2;
-constexpr int kThreads = 32 * (kComputeWarps + 3);
-constexpr int kRowStride = 64;                        // unrotated mapping: rows t/8 and t/8 + 64
+// Warps 16-19 (TMEM lane quadrants 0-3) read out L; 16 and 17 first run the
+// producer (with the stores) and the MMAs.  (Twenty warps: registers are allocated for
+// blocks in groups of four warps, so a 21st would cost the 96-register budget.)
+constexpr int kProducerWarp = kComputeWarps, kMmaWarp = kComputeWarps + 1, kLrWarp0 = kComputeWarps;
+constexpr int kThreads = 32 * (kComputeWarps + 4);
+// Unrotated mapping: thread t takes block column t % 8 of rows t/8 + kRowStride * i.
+constexpr int kRowStride = kComputeThreads / 8;
+constexpr int kRowsPerThread = kRows / kRowStride;
+// Rotated mapping: four threads per row, kRotPasses rows per thread in turn.
+constexpr int kRotRowsPerPass = kComputeThreads / 4;
+constexpr int kRotPasses = kRows / kRotRowsPerPass;
 
 struct QParams {
   const float4* lamq;       // smoothing reciprocal pairs, lam_slot order
@@ -136,7 +149,7 @@ __device__ __forceinline__ uint32_t quant_block_rr(const uint64_t (&v)[8], float
   return sb;
 }
 
-// x / smooth for 16 channels (bf16 words xin) with the IEEE divide: the path
+// x / smooth for 2N channels (bf16 words xin) with the IEEE divide: the path
 // for blocks whose fast quotients overflowed or hold NaN.
 template <int N>
 __device__ __forceinline__ void smooth_ieee(const uint32_t (&xin)[N], const float* lamf, int k, uint64_t (&v)[N]) {
@@ -146,6 +159,22 @@ __device__ __forceinline__ void smooth_ieee(const uint32_t (&xin)[N], const floa
                __fdiv_rn(__uint_as_float(xin[i] & 0xFFFF0000u), lamf[k + 2 * i + 1]));
 }
 
+// The IEEE path of one unrotated block (values that overflowed or hold NaN),
+// out of line so that the rare path stays out of the hot loop's instruction
+// stream: it reloads the block's x from shared memory and returns the codes
+// and the scale byte by value (passing the caller's register arrays would put
+// them in local memory on the fast path too).
+__device__ __noinline__ uint3 smooth_quant_block_ieee(const uint8_t* xs, int row, int j, const float* lamf, int k) {
+  const uint4 p0 = *reinterpret_cast<const uint4*>(xs + xoff(row, 2 * j));
+  const uint4 p1 = *reinterpret_cast<const uint4*>(xs + xoff(row, 2 * j + 1));
+  const uint32_t xin[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+  uint64_t v[8];
+  smooth_ieee(xin, lamf, k, v);
+  uint3 r;
+  r.z = quant_block_slow(v, r.x, r.y);
+  return r;
+}
+
 // Unrotated path, one thread: 16-channel block column j = t & 7 of the chunk
 // for rows t/8 and t/8 + 64; the block's smoothing operands are read once for
 // both rows.  Rows at or beyond `nvalid` (zero-filled by the TMA) get zero
@@ -153,12 +182,12 @@ __device__ __forceinline__ void smooth_ieee(const uint32_t (&xin)[N], const floa
 template <bool FULL>
 __device__ __forceinline__ void smooth_rows(const uint8_t* xs, const float4* lam, const float2* srec, float yh6,
                                             float yl6, const float* lamf, int kc, int t, int nvalid,
-                                            uint32_t (&cw)[2][2], uint32_t (&sb)[2]) {
+                                            uint32_t (&cw)[kRowsPerThread][2], uint32_t (&sb)[kRowsPerThread]) {
   const int j = t & 7, r0 = t >> 3;
-  bool live[2];
-  uint32_t xin[2][8];
+  bool live[kRowsPerThread];
+  uint32_t xin[kRowsPerThread][8];
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
+  for (int rr = 0; rr < kRowsPerThread; ++rr) {
     const int row = r0 + kRowStride * rr;
     live[rr] = FULL || row < nvalid;
     if (live[rr]) {
@@ -171,23 +200,25 @@ __device__ __forceinline__ void smooth_rows(const uint8_t* xs, const float4* lam
       for (int i = 0; i < 8; ++i) xin[rr][i] = 0u;
     }
   }
-  uint64_t v[2][8];
+  uint64_t v[kRowsPerThread][8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float4 l = lam[8 * i + j];                  // pair 8j + i (see lam_slot)
     const uint64_t yh = pk2(l.x, l.y), yl = pk2(l.z, l.w);
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr) v[rr][i] = div_rr2(bf16x2_to_f2(xin[rr][i]), yh, yl);
+    for (int rr = 0; rr < kRowsPerThread; ++rr) v[rr][i] = div_rr2(bf16x2_to_f2(xin[rr][i]), yh, yl);
   }
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
+  for (int rr = 0; rr < kRowsPerThread; ++rr) {
     const float amax = amax8(v[rr]);
     if (amax < 3.0e38f) {
       sb[rr] = quant_block_rr(v[rr], amax, srec, yh6, yl6, cw[rr][0], cw[rr][1]);
     } else {
       // A block holds +-inf or NaN, or overflowed (rare): the divide unit.
-      smooth_ieee(xin[rr], lamf, kc + 16 * j, v[rr]);
-      sb[rr] = quant_block_slow(v[rr], cw[rr][0], cw[rr][1]);
+      const uint3 r = smooth_quant_block_ieee(xs, r0 + kRowStride * rr, j, lamf, kc + 16 * j);
+      cw[rr][0] = r.x;
+      cw[rr][1] = r.y;
+      sb[rr] = r.z;
     }
     if (!live[rr]) {
       cw[rr][0] = cw[rr][1] = 0u;
@@ -196,11 +227,11 @@ __device__ __forceinline__ void smooth_rows(const uint8_t* xs, const float4* lam
   }
 }
 
-__device__ __forceinline__ void stage_rows(uint8_t* cst, uint8_t* sst, int t, const uint32_t (&cw)[2][2],
-                                           const uint32_t (&sb)[2]) {
+__device__ __forceinline__ void stage_rows(uint8_t* cst, uint8_t* sst, int t, const uint32_t (&cw)[kRowsPerThread][2],
+                                           const uint32_t (&sb)[kRowsPerThread]) {
   const int j = t & 7, r0 = t >> 3;
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
+  for (int rr = 0; rr < kRowsPerThread; ++rr) {
     const int row = r0 + kRowStride * rr;
     *reinterpret_cast<uint2*>(cst + row * (kChunk / 2) + j * 8) = make_uint2(cw[rr][0], cw[rr][1]);
     sst[(j >> 2) * kSfAtomBytes + sf_atom_offset(row, j & 3)] = (uint8_t)sb[rr];
@@ -208,13 +239,13 @@ __device__ __forceinline__ void stage_rows(uint8_t* cst, uint8_t* sst, int t, co
 }
 
 // Row-major (caller layout) stores of the unrotated mapping.
-__device__ __forceinline__ void store_rows(const QParams& p, int m0, int t, int kc, const uint32_t (&cw)[2][2],
-                                           const uint32_t (&sb)[2]) {
+__device__ __forceinline__ void store_rows(const QParams& p, int m0, int t, int kc,
+                                           const uint32_t (&cw)[kRowsPerThread][2], const uint32_t (&sb)[kRowsPerThread]) {
   const int j = t & 7, r0 = t >> 3;
   const int k = kc + 16 * j;
   if (k >= p.k_limit) return;
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
+  for (int rr = 0; rr < kRowsPerThread; ++rr) {
     const int m = m0 + r0 + kRowStride * rr;
     if (m >= p.M) continue;
     *reinterpret_cast<uint2*>(p.codes + (size_t)m * p.codes_pitch + (k >> 1)) = make_uint2(cw[rr][0], cw[rr][1]);
@@ -302,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(tabs + 1);
   uint64_t* full = bars;                     // TMA landed
   uint64_t* cdone = bars + p.stages;         // compute threads finished the stage (512 arrivals)
-  uint64_t* empty = bars + 2 * p.stages;     // MMA read + stores read the stage (2 arrivals)
+  uint64_t* empty = bars + 2 * p.stages;     // the MMAs have read the stage
   uint64_t* done = bars + 3 * p.stages;      // all MMAs of this CTA finished
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * p.stages + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -317,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&cdone[s]), kComputeThreads);
-      mbar_init(smem_u32(&empty[s]), 2);
+      mbar_init(smem_u32(&empty[s]), 1);
     }
     mbar_init(smem_u32(done), 1);
     *abort_flag = 0;
@@ -347,11 +378,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   int issued = 0;   // producer: loads issued
   if (warp == kProducerWarp) {
     if (lane == 0) {
-      for (int i = 0; i < nch; ++i) {
+      auto load = [&](int i) {
         const int s = i % p.stages;
-        if (i >= p.stages &&
-            !wait_bounded(smem_u32(&empty[s]), ((i / p.stages) - 1) & 1, abort_flag, p.err, kErrQuantTimeout))
-          break;
         const int kc = (c_begin + i) * kChunk;
         const uint32_t fb = smem_u32(&full[s]);
         mbar_arrive_expect_tx(fb, kXStageBytes + pd_stage_bytes + kLamStageBytes);
@@ -363,7 +391,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(smem_u32(pds + R * 128), &tm_pdT, fb, kc + 64, 0);
         bulk_load(smem_u32(LAM + s * kLamStageBytes), p.lamq + kc / 2, kLamStageBytes, fb);
         issued = i + 1;
+      };
+      for (int i = 0; i < nch && i < p.stages; ++i) load(i);
+      for (int j = 0; j < nch; ++j) {
+        const int s = j % p.stages, par = (j / p.stages) & 1;
+        // Chunk j's codes and scales are staged: write them.
+        if (!wait_bounded(smem_u32(&cdone[s]), par, abort_flag, p.err, kErrQuantTimeout)) break;
+        if (TILED) {
+          const int kc = (c_begin + j) * kChunk;
+          tma_store_2d(&tm_codes, smem_u32(CST + s * kCodeStageBytes), kc / 2, m0);
+          bulk_store(p.scales + ((size_t)blockIdx.x * p.ka_pad + kc / 64) * kSfAtomBytes,
+                     smem_u32(SST + s * kSfStageBytes), kSfStageBytes);
+          bulk_commit();
+        }
+        if (j + p.stages < nch) {
+          // The stage is reused once the stores and the MMAs have read it.
+          if (TILED) bulk_wait_read<0>();
+          if (!wait_bounded(smem_u32(&empty[s]), par, abort_flag, p.err, kErrQuantTimeout)) break;
+          load(j + p.stages);
+        }
       }
+      // The staging buffers have been read; the stores themselves complete
+      // at the end, after this warp's share of the rank-R read-out.
+      if (TILED) bulk_wait_read<0>();
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -388,32 +438,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(smem_u32(done));
     }
     __syncwarp();
-  } else if (warp == kStoreWarp) {
-    if (lane == 0) {
-      for (int i = 0; i < nch; ++i) {
-        const int s = i % p.stages;
-        if (!wait_bounded(smem_u32(&cdone[s]), (i / p.stages) & 1, abort_flag, p.err, kErrQuantTimeout)) break;
-        if (TILED) {
-          // Every compute thread has staged its codes and scales: write the
-          // chunk's code tile and its two adjacent scale atoms, and release
-          // the stage once they have been read.
-          const int kc = (c_begin + i) * kChunk;
-          tma_store_2d(&tm_codes, smem_u32(CST + s * kCodeStageBytes), kc / 2, m0);
-          bulk_store(p.scales + ((size_t)blockIdx.x * p.ka_pad + kc / 64) * kSfAtomBytes,
-                     smem_u32(SST + s * kSfStageBytes), kSfStageBytes);
-          bulk_commit();
-          bulk_wait_read<0>();
-        }
-        mbar_arrive(smem_u32(&empty[s]));
-      }
-      if (TILED) bulk_wait<0>();
-    }
-    __syncwarp();
-  } else {
+  } else if (warp < kComputeWarps) {
     // compute warps: the chunk's 128 rows x 128 channels
     const float2 r6 = recip_pair(6.0f);
     const float yh6 = r6.x, yl6 = r6.y;
-    const int row4 = tid >> 2, qq = tid & 3;     // rotated mapping: four threads per row
+    const int row4 = tid >> 2, qq = tid & 3;     // rotated mapping: four threads per row (first pass)
     const int nvalid = p.M - m0;                 // rows of this tile that exist (>= 1)
     for (int i = 0; i < nch; ++i) {
       const int s = i % p.stages;
@@ -424,17 +453,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int kc = (c_begin + i) * kChunk;
       const uint8_t* xs = X + s * kXStageBytes;
       const float4* lam = reinterpret_cast<const float4*>(LAM + s * kLamStageBytes);
-      uint32_t cwq[4], sq = 0u;                                     // rotated mapping
-      uint32_t cw[2][2], sb[2];                                     // column mapping
+      uint32_t cwq[kRotPasses][4], sq[kRotPasses];                  // rotated mapping
+      uint32_t cw[kRowsPerThread][2], sb[kRowsPerThread];           // column mapping
       if (ROT) {
         // Only a whole warp may skip (full-warp shuffles): all 8 of its rows
         // lie beyond M.  Rows beyond M that a warp does process are
         // zero-filled and rotate to zero.
-        if ((row4 & ~7) < nvalid) {
-          rotate_quarter(xs, lam, tabs->srec, yh6, yl6, p.lamf, kc, row4, qq, cwq, sq);
-        } else {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) cwq[c] = 0u;
+        for (int ps = 0; ps < kRotPasses; ++ps) {
+          sq[ps] = 0u;
+          if ((row4 & ~7) + kRotRowsPerPass * ps < nvalid) {
+            rotate_quarter(xs, lam, tabs->srec, yh6, yl6, p.lamf, kc, row4 + kRotRowsPerPass * ps, qq, cwq[ps], sq[ps]);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) cwq[ps][c] = 0u;
+          }
         }
       } else if (nvalid >= kRows) {
         smooth_rows<true>(xs, lam, tabs->srec, yh6, yl6, p.lamf, kc, tid, nvalid, cw, sb);
@@ -446,13 +479,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         // before the stage was released for this chunk's load.
         uint8_t* cst = CST + s * kCodeStageBytes;
         uint8_t* sst = SST + s * kSfStageBytes;
-        if (ROT)
-          stage_quarter(cst, sst, row4, qq, cwq, sq);
-        else
+        if (ROT) {
+#pragma unroll
+          for (int ps = 0; ps < kRotPasses; ++ps) stage_quarter(cst, sst, row4 + kRotRowsPerPass * ps, qq, cwq[ps], sq[ps]);
+        } else {
           stage_rows(cst, sst, tid, cw, sb);
+        }
       } else if (ROT) {
-        const int m = m0 + row4, k0 = kc + 32 * qq;
-        if (m < p.M && k0 < p.k_limit) store_quarter(p, m, k0, cwq, sq);
+#pragma unroll
+        for (int ps = 0; ps < kRotPasses; ++ps) {
+          const int m = m0 + row4 + kRotRowsPerPass * ps, k0 = kc + 32 * qq;
+          if (m < p.M && k0 < p.k_limit) store_quarter(p, m, k0, cwq[ps], sq[ps]);
+        }
       } else {
         store_rows(p, m0, tid, kc, cw, sb);
       }
@@ -477,12 +515,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // order (a fixed order: the result does not depend on timing).
   const bool want_lr = p.lowrank != nullptr;
   const int rows_per = kRows / p.ksplit;
-  if (want_lr && tid < kRows) {
-    // warps 0-3 read TMEM lane quadrants 0-3: thread tid owns row tid.
+  if (want_lr && warp >= kLrWarp0 && warp < kLrWarp0 + 4) {
+    // Warps 16-19 read TMEM lane quadrants 0-3 (warp % 4): lane l of warp w
+    // owns row 32 (w % 4) + l.  This runs as soon as the last MMA has
+    // completed, while the compute warps may still be on their last chunks.
     // Warp-uniform outcome: the TMEM loads below are warp-wide instructions.
     const bool ok = __all_sync(0xffffffffu, wait_bounded(smem_u32(done), 0, abort_flag, p.err, kErrQuantTimeout));
     tc_fence_after_sync();
-    const int row = tid, m = m0 + row;
+    const int row = 32 * (warp & 3) + lane, m = m0 + row;
     const uint32_t owner = (uint32_t)(row / rows_per);
     const uint32_t dst0 = p.ksplit > 1 ? mapa_shared(smem_u32(recv) + (uint32_t)(((int)cluster_ctarank() * rows_per +
                                                                                   row % rows_per) * R * 4),
@@ -491,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       for (int j = 0; j < R; j += 16) {
         uint32_t r[16];
-        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)j, r);
+        tmem_ld16(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)j, r);
         tmem_ld_wait();
         if (p.ksplit == 1) {
           if (m < p.M) {
@@ -546,6 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   if (warp == kMmaWarp && lane == 0) wait_for(smem_u32(done), 0, kWaitTimeoutNs);
+  if (TILED && warp == kProducerWarp && lane == 0) bulk_wait<0>();
   tc_fence_before_sync();
   __syncthreads();
   if (warp == kProducerWarp) {

@@ -48,6 +48,10 @@ struct MxQuantLaunch {
 };
 cudaError_t launch_quantize_mx(const MxQuantLaunch& p, cudaStream_t stream);
 
+// Back-to-back block-scaled FP4 MMAs on `ctas` CTAs (one per SM), operands in
+// shared memory: the measured dense FP4 tensor rate.
+cudaError_t launch_fp4_mma_loop(int iters, int ctas, unsigned* err, cudaStream_t stream);
+
 // Standalone Walsh-Hadamard transform of rows of length 2^log2n (<= 2^15),
 // in place; dtype 0 = bf16, 1 = fp16.
 cudaError_t launch_hadamard_transform(void* x, int rows, int log2n, int dtype, cudaStream_t stream);

@@ -322,6 +322,21 @@ SVDQ_API svdq_status svdq_mxfp4_forward(const svdq_mxfp4* h, const void* x, int 
 /* As svdq_device_status, for an MXFP4 handle (bit 1: the GEMM's bounded wait expired). */
 SVDQ_API svdq_status svdq_mxfp4_device_status(const svdq_mxfp4* h, int* flags);
 
+/*
+ * svdq_fp4_mma_loop -- a measurement utility, with no counterpart in the pages:
+ * the dense block-scaled FP4 tensor-core rate of the current device, which the
+ * GEMM's roofline fraction divides by.  Launches one CTA per SM on `stream`;
+ * each issues `iters` x 4 back-to-back tcgen05.mma kind::mxf4nvf4 (NVFP4,
+ * M = 128, N = 256, K = 64) from shared memory with no loads in the loop.
+ * *ctas receives the number of CTAs; the launch performs
+ * (*ctas) * iters * 4 * 2 * 128 * 256 * 64 flops.  Time it with CUDA events on
+ * `stream`.  1 <= iters <= 2^20 (at most about a quarter of a second).
+ * svdq_fp4_mma_loop_status synchronizes the device and reads + clears the
+ * loop's error word (nonzero when its bounded wait expired).
+ */
+SVDQ_API svdq_status svdq_fp4_mma_loop(int iters, int* ctas, void* stream);
+SVDQ_API svdq_status svdq_fp4_mma_loop_status(int* flags);
+
 /* Static text for a status code. */
 SVDQ_API const char* svdq_status_string(svdq_status s);
 

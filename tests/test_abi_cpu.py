@@ -23,7 +23,8 @@ def test_exports_every_declared_symbol(lib):
         "svdq_last_error", "svdq_version", "svdq_linear_forward_quantize", "svdq_linear_forward_gemm",
         "svdq_linear_forward_noalloc", "svdq_quantize_weight", "svdq_hadamard_transform",
         "svdq_linear_gemm_kernel", "svdq_mxfp4_create", "svdq_mxfp4_destroy", "svdq_mxfp4_workspace_bytes",
-        "svdq_mxfp4_quantize", "svdq_mxfp4_forward", "svdq_mxfp4_device_status"}
+        "svdq_mxfp4_quantize", "svdq_mxfp4_forward", "svdq_mxfp4_device_status", "svdq_fp4_mma_loop",
+        "svdq_fp4_mma_loop_status"}
     for n in names:
         assert hasattr(lib, n), n
 
@@ -140,3 +141,9 @@ def test_mxfp4_quantize_rejects_bad_args_on_host(lib):
     assert lib.svdq_mxfp4_quantize(16, 0, 64, 32, 16, 16, None) == 0     # M == 0: no-op
     assert lib.svdq_mxfp4_workspace_bytes(None, 4) == 0
     assert lib.svdq_mxfp4_forward(None, 16, 4, 16, 256, None) == 1
+
+
+def test_fp4_loop_rejects_bad_iters_on_host(lib):
+    ctas = ctypes.c_int(-1)
+    assert lib.svdq_fp4_mma_loop(0, ctypes.byref(ctas), None) == 1
+    assert lib.svdq_fp4_mma_loop((1 << 20) + 1, ctypes.byref(ctas), None) == 1
