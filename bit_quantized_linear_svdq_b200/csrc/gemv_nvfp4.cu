@@ -56,7 +56,9 @@ struct GvParams {
   const uint8_t* sfr;      // (N, Kp/16) weight block scales, row-major e4m3
   const uint8_t* codes;    // (M, Kp/2) activation codes
   const uint8_t* sfa;      // activation scale atoms (row tile 0)
-  const __nv_bfloat16* lowrank;   // (M, R)
+  const __nv_bfloat16* lowrank;   // (M, R), when lr_part is null
+  const float* lr_part;           // [n_parts][M][R] fp32 partial L, or null
+  int n_parts;
   const __nv_bfloat16* pu;        // (N, R)
   const float* alpha;             // (N)
   __nv_bfloat16* y;               // (M, N)
@@ -134,8 +136,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_nvfp4_kernel(const GvParams 
   if (tid == 0) griddep_launch_dependents();
 
   // Token rows -> shared memory: codes as fp16 (8 per 4-byte word), block
-  // scales as fp32 (zero for blocks at or beyond K), L as fp32.
-  for (int i = tid; i < MT * (kgrp / 8); i += kThreads) {
+  // scales as fp32 (zero for blocks at or beyond K), L as fp32.  Every
+  // thread issues its loads of all three first, so their latencies overlap.
+  constexpr int kCodeIters = 2, kScaleIters = 1;           // loads issued up front; any remainder uses plain loops
+  uint32_t cw[kCodeIters];
+  uint32_t sbv[kScaleIters];
+#pragma unroll
+  for (int c = 0; c < kCodeIters; ++c) {
+    const int i = tid + c * kThreads;
+    const int m = i / (kgrp / 8), k = (i % (kgrp / 8)) * 8;
+    cw[c] = (i < MT * (kgrp / 8) && m < p.M && k < p.K) ? __ldg(reinterpret_cast<const uint32_t*>(p.codes + (size_t)m * rb + k / 2)) : 0u;
+  }
+#pragma unroll
+  for (int c = 0; c < kScaleIters; ++c) {
+    const int i = tid + c * kThreads;
+    const int m = i / sb, kb = i % sb;
+    sbv[c] = (i < MT * sb && m < p.M && kb < K16) ? p.sfa[(size_t)(kb >> 2) * kSfAtomBytes + sf_atom_offset(m, kb & 3)] : 0xFFFFFFFFu;
+  }
+  for (int i = tid + kCodeIters * kThreads; i < MT * (kgrp / 8); i += kThreads) {   // larger K: the plain loop
     const int m = i / (kgrp / 8), k = (i % (kgrp / 8)) * 8;
     uint4 o = make_uint4(0u, 0u, 0u, 0u);
     if (m < p.M && k < p.K) {
@@ -145,16 +163,48 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_nvfp4_kernel(const GvParams 
     }
     *reinterpret_cast<uint4*>(act + m * kgrp + act_slot(k)) = o;
   }
-  for (int i = tid; i < MT * sb; i += kThreads) {
+  for (int i = tid + kScaleIters * kThreads; i < MT * sb; i += kThreads) {
     const int m = i / sb, kb = i % sb;
     float v = 0.0f;
-    if (m < p.M && kb < K16)
-      v = e4m3_to_f(p.sfa[(size_t)(kb >> 2) * kSfAtomBytes + sf_atom_offset(m, kb & 3)]);
+    if (m < p.M && kb < K16) v = e4m3_to_f(p.sfa[(size_t)(kb >> 2) * kSfAtomBytes + sf_atom_offset(m, kb & 3)]);
     sa[i] = v;
   }
-  for (int i = tid; i < MT * p.R; i += kThreads) {
-    const int m = i / p.R;
-    lr[i] = m < p.M ? __bfloat162float(p.lowrank[i]) : 0.0f;
+  if (p.lr_part) {
+    // The few-row quantizer's per-slice partial sums of L: sixteen threads
+    // per (row, rank) each add the slices s = sub, sub + 16, ... in order,
+    // then a fixed shuffle tree adds the sixteen (deterministic), so every
+    // load is in flight at once.
+    for (int i0 = 0; i0 < MT * p.R; i0 += kThreads / 16) {
+      const int i = i0 + (tid >> 4), sub = tid & 15;
+      const int m = i / p.R, r = i % p.R;
+      float v = 0.0f;
+      if (i < MT * p.R && m < p.M)
+        for (int s = sub; s < p.n_parts; s += 16) v += __ldg(p.lr_part + ((size_t)s * p.M + m) * p.R + r);
+#pragma unroll
+      for (int o = 8; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (sub == 0 && i < MT * p.R) lr[i] = v;
+    }
+  } else {
+    for (int i = tid; i < MT * p.R; i += kThreads) {
+      const int m = i / p.R;
+      lr[i] = m < p.M ? __bfloat162float(p.lowrank[i]) : 0.0f;
+    }
+  }
+  // The first iterations' values, loaded above.
+#pragma unroll
+  for (int c = 0; c < kCodeIters; ++c) {
+    const int i = tid + c * kThreads;
+    if (i < MT * (kgrp / 8)) {
+      const int m = i / (kgrp / 8), k = (i % (kgrp / 8)) * 8;
+      uint32_t d[4];
+      e2m1x8_to_f16x8(cw[c], d);
+      *reinterpret_cast<uint4*>(act + m * kgrp + act_slot(k)) = make_uint4(d[0], d[1], d[2], d[3]);
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < kScaleIters; ++c) {
+    const int i = tid + c * kThreads;
+    if (i < MT * sb) sa[i] = sbv[c] == 0xFFFFFFFFu ? 0.0f : e4m3_to_f(sbv[c]);
   }
   __syncthreads();
 
@@ -270,6 +320,8 @@ cudaError_t launch_gemv_nvfp4(const GemvLaunch& L, cudaStream_t stream) {
   p.codes = L.codes;
   p.sfa = L.sfa;
   p.lowrank = static_cast<const __nv_bfloat16*>(L.lowrank);
+  p.lr_part = L.lr_part;
+  p.n_parts = L.n_parts;
   p.pu = static_cast<const __nv_bfloat16*>(L.pu);
   p.alpha = L.alpha;
   p.y = static_cast<__nv_bfloat16*>(L.y);

@@ -279,15 +279,20 @@ void free_handle(svdq_linear* h) {
 }
 
 struct WsLayout {
-  size_t codes, sfa, lr, total;
+  size_t codes, sfa, lr, part, total;
 };
 
+// Workspace of one call: codes, scale atoms, L (bf16), and for at most
+// kGemvMaxRows rows the few-row quantizer's fp32 partial L per 128-channel slice.
 WsLayout ws_layout(const svdq_linear* h, int M) {
   WsLayout w;
   w.codes = 0;
   w.sfa = align256((size_t)M * (h->Kp / 2));
   w.lr = align256(w.sfa + (size_t)((M + 127) / 128) * h->ka_pad * svdq::kSfAtomBytes);
-  w.total = align256(w.lr + (size_t)M * h->R * 2);
+  w.part = align256(w.lr + (size_t)M * h->R * 2);
+  const size_t part_bytes =
+      M <= svdq::kGemvMaxRows ? (size_t)svdq::quantize_few_slices(h->Kp) * M * h->R * sizeof(float) : 0;
+  w.total = align256(w.part + part_bytes);
   return w;
 }
 
@@ -526,9 +531,34 @@ svdq_status check_forward_args(const svdq_linear* h, int M, void* workspace) {
   return check_device(h);
 }
 
+enum class GemmKind { gemv, narrow, splitk, pair, n256, lr };
+GemmKind pick_gemm(const svdq_linear* h, int M, int* S);
+
 svdq_status forward_quantize(const svdq_linear* h, const void* x, int M, void* workspace, cudaStream_t stream) {
   const WsLayout w = ws_layout(h, M);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int S = 1;
+  if (pick_gemm(h, M, &S) == GemmKind::gemv) {
+    // 1..4 rows on the CUDA-core matrix-vector product: its own quantizer
+    // (codes, scale atoms, per-slice partial L), no tensor-core tiles.
+    svdq::FewQuantLaunch f;
+    f.x = x;
+    f.lamq = h->lamq;
+    f.lamf = h->lamf;
+    f.pdT = h->pdT;
+    f.codes = ws + w.codes;
+    f.sfa = ws + w.sfa;
+    f.part = reinterpret_cast<float*>(ws + w.part);
+    f.M = M;
+    f.K = h->K;
+    f.Kp = h->Kp;
+    f.R = h->R;
+    f.ka_pad = h->ka_pad;
+    f.rotate_block = h->rotate_block;
+    cudaError_t e = svdq::launch_quantize_few(f, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "quantize_few launch");
+    return SVDQ_OK;
+  }
   svdq::QuantLaunch q;
   svdq_status s;
   if ((s = make_tmap(&q.tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, h->K, M, (uint64_t)h->K * 2, 64, 128)) != SVDQ_OK)
@@ -570,7 +600,6 @@ int num_sms() {
 }
 
 // Which GEMM kernel serves M rows on this handle (S: split-K cluster size).
-enum class GemmKind { gemv, narrow, splitk, pair, n256, lr };
 
 GemmKind pick_gemm(const svdq_linear* h, int M, int* S) {
   *S = 1;
@@ -598,6 +627,8 @@ svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, 
     v.codes = ws + w.codes;
     v.sfa = ws + w.sfa;
     v.lowrank = ws + w.lr;
+    v.lr_part = reinterpret_cast<const float*>(ws + w.part);
+    v.n_parts = svdq::quantize_few_slices(h->Kp);
     v.pu = h->pu;
     v.alpha = h->alpha;
     v.y = y;

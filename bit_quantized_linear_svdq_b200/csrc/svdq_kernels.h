@@ -116,12 +116,31 @@ bool gemm_narrow_applies(int M, int R);
 // of the weight block scales (N, Kp/16), the activation codes and scale atoms
 // the quantizer wrote, L (M, R), proj_up (N, R), the plain alpha (N).
 constexpr int kGemvMaxRows = 4;
+// The activation quantizer for 1..kGemvMaxRows rows on CUDA cores: one CTA
+// per 128-channel slice writes codes (M, Kp/2), the scale atoms of row tile 0
+// and the slice's fp32 partial L = x P into part[slice][M][R]; the
+// matrix-vector kernel adds the partials in slice order.
+struct FewQuantLaunch {
+  const void* x;            // bf16 (M, K)
+  const void* lamq;         // as QuantLaunch
+  const float* lamf;
+  const void* pdT;          // P^T bf16 (R, Kp)
+  uint8_t* codes;
+  uint8_t* sfa;
+  float* part;
+  int M, K, Kp, R, ka_pad, rotate_block;
+};
+cudaError_t launch_quantize_few(const FewQuantLaunch& p, cudaStream_t stream);
+int quantize_few_slices(int Kp);
+
 struct GemvLaunch {
   const uint8_t* qw;
   const uint8_t* sfr;
   const uint8_t* codes;
   const uint8_t* sfa;
-  const void* lowrank;
+  const void* lowrank;      // (M, R) bf16, used when lr_part is null
+  const float* lr_part;     // [n_parts][M][R] fp32 partial L (the few-row quantizer's), or null
+  int n_parts;
   const void* pu;
   const float* alpha;
   void* y;
