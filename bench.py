@@ -344,7 +344,6 @@ def run_ours(args, world, rank, local):
         sets.append((layer, x, y, ws))
     stream = torch.cuda.Stream()
     variant = sets[0][0].gemm_kernel(M)
-    gemm_bound = "hbm" if variant.startswith("gemv") else "tensor"
 
     def step(i, which="both"):
         layer, x, y, ws = sets[i % N_SETS]
@@ -504,6 +503,9 @@ def run_ours(args, world, rank, local):
     q_gbs = quant_bytes(M, K, R) / (us_q * 1e-6) / 1e9
     g_flops = 2.0 * M * N * K + 2.0 * M * N * R
     g_tf = g_flops / (us_g * 1e-6) / 1e12
+    # The GEMM's roofline bound: the slower of its flops at the FP4 peak and
+    # its bytes at HBM bandwidth (few rows: the weight read).
+    gemm_bound = "hbm" if gemm_bytes(M, K, N, R) / (pk["hbm_gbs"] * 1e9) > g_flops / (fp4_peak * 1e12) else "tensor"
     kernels = {
         "quantize_act": {"us": us_q, "bound": "hbm", "algorithmic_bytes": quant_bytes(M, K, R),
                          "achieved_gbs": q_gbs, "frac_of_hbm": q_gbs / pk["hbm_gbs"],
