@@ -99,6 +99,131 @@ __device__ __forceinline__ float f16x2_sum(uint32_t v) {
   return f.x + f.y;
 }
 
+// One pass of 16-byte weight pieces of row n (and their two block-scale
+// bytes each); zeros past N or the row's end.
+__device__ __forceinline__ void load_pass(const GvParams& p, int n, int pass, int lane, uint4 (&v)[kPieces],
+                                          uint32_t (&s)[kPieces]) {
+  const int pieces = p.Kp / 32, rb = p.Kp / 2, sb = p.Kp / 16;
+#pragma unroll
+  for (int j = 0; j < kPieces; ++j) {
+    const int u = pass * kPass + j * 32 + lane;
+    if (n < p.N && u < pieces) {
+      v[j] = __ldg(reinterpret_cast<const uint4*>(p.qw + (size_t)n * rb) + u);
+      s[j] = __ldg(reinterpret_cast<const unsigned short*>(p.sfr + (size_t)n * sb) + u);
+    } else {
+      v[j] = make_uint4(0u, 0u, 0u, 0u);
+      s[j] = 0u;
+    }
+  }
+}
+
+// A warp's first two weight rows (first pass), their proj_up entries (rank
+// r = lane) and alpha.  All are library-owned weights written at create
+// (which synchronizes), so they are requested before the dependency wait and
+// stream in while the previous kernel is still running.
+struct RowPrefetch {
+  uint4 wv[2][kPieces];
+  uint32_t ws2[2][kPieces];
+  float pu[2], al[2];
+};
+
+__device__ __forceinline__ void prefetch_rows(const GvParams& p, int w0, int W, int lane, RowPrefetch& f) {
+  load_pass(p, w0, 0, lane, f.wv[0], f.ws2[0]);
+  load_pass(p, w0 + W, 0, lane, f.wv[1], f.ws2[1]);
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int n = w0 + r * W;
+    f.pu[r] = 0.0f;
+    f.al[r] = 0.0f;
+    if (n < p.N) {
+      if (lane < p.R) f.pu[r] = __bfloat162float(p.pu[(size_t)n * p.R + lane]);
+      f.al[r] = __ldg(p.alpha + n);
+    }
+  }
+}
+
+// The product for the warp's weight rows w0, w0 + W, ... (two at a time),
+// from the token rows in shared memory: act (fp16, act_slot order, kgrp
+// slots per row), sa (fp32 block scales, Kp/16 per row) and lr (L, R per row).
+template <int MT>
+__device__ __forceinline__ void dot_rows(const GvParams& p, const uint16_t* act, const float* sa, const float* lr,
+                                         int kgrp, int w0, int W, int lane, RowPrefetch& f) {
+  const int pieces = p.Kp / 32, sb = p.Kp / 16;
+  const int passes = (pieces + kPass - 1) / kPass;
+  for (int n0 = w0; n0 < p.N; n0 += 2 * W) {
+    float acc[2][MT];
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) acc[r][m] = 0.0f;
+    for (int pass = 0; pass < passes; ++pass) {
+      if (n0 != w0 || pass != 0) {
+        load_pass(p, n0, pass, lane, f.wv[0], f.ws2[0]);
+        load_pass(p, n0 + W, pass, lane, f.wv[1], f.ws2[1]);
+      }
+#pragma unroll
+      for (int j = 0; j < kPieces; ++j) {
+        const int u = pass * kPass + j * 32 + lane;
+        if (u >= pieces) break;
+        const int k0 = 32 * u;
+        const uint4* ap = reinterpret_cast<const uint4*>(act + act_slot(k0));
+        float2 sav[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) sav[m] = *reinterpret_cast<const float2*>(sa + m * sb + 2 * u);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const uint32_t wb[4] = {f.wv[r][j].x, f.wv[r][j].y, f.wv[r][j].z, f.wv[r][j].w};
+          uint32_t wf[4][4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) e2m1x8_to_f16x8(wb[q], wf[q]);
+          const float2 sw = make_float2(e4m3_to_f(f.ws2[r][j] & 0xFF), e4m3_to_f(f.ws2[r][j] >> 8));
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            uint32_t h0 = 0u, h1 = 0u;                       // +0.0 in both halves
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 a = ap[m * (kgrp / 8) + q * 32];
+              const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+              for (int b = 0; b < 4; ++b) {
+                if (q < 2) h0 = hfma2(wf[q][b], av[b], h0);
+                else h1 = hfma2(wf[q][b], av[b], h1);
+              }
+            }
+            acc[r][m] = fmaf(f16x2_sum(h0), sav[m].x * sw.x, acc[r][m]);
+            acc[r][m] = fmaf(f16x2_sum(h1), sav[m].y * sw.y, acc[r][m]);
+          }
+        }
+      }
+    }
+    // Rank-R term, then the warp reductions (fixed tree) and the store.
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int n = n0 + r * W;
+      if (n >= p.N) break;                                 // warp-uniform
+      const float al = n0 == w0 ? f.al[r] : p.alpha[n];
+      float l[MT];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) l[m] = 0.0f;
+      for (int rr = lane; rr < p.R; rr += 32) {
+        const float pv = (n0 == w0 && rr == lane) ? f.pu[r] : __bfloat162float(p.pu[(size_t)n * p.R + rr]);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) l[m] = fmaf(lr[m * p.R + rr], pv, l[m]);
+      }
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        float a = acc[r][m], b = l[m];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+          a += __shfl_xor_sync(0xffffffffu, a, o);
+          b += __shfl_xor_sync(0xffffffffu, b, o);
+        }
+        if (lane == m && m < p.M) p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(fmaf(al, a, b));
+      }
+    }
+  }
+}
+
 template <int MT>
 __global__ void __launch_bounds__(kThreads, 1) gemv_nvfp4_kernel(const GvParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
@@ -109,28 +234,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_nvfp4_kernel(const GvParams 
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int W = gridDim.x * kWarps, w0 = blockIdx.x * kWarps + warp;
-  const int pieces = p.Kp / 32;                             // 16-byte pieces per row
   const int rb = p.Kp / 2, sb = p.Kp / 16;                  // row bytes: codes, scales
   const int K16 = p.K / 16;
 
-  // First two rows, first pass: requested before the dependency wait.
-  uint4 wv[2][kPieces];
-  uint32_t ws2[2][kPieces];
-  auto load_pass = [&](int n, int pass, uint4 (&v)[kPieces], uint32_t (&s)[kPieces]) {
-#pragma unroll
-    for (int j = 0; j < kPieces; ++j) {
-      const int u = pass * kPass + j * 32 + lane;
-      if (n < p.N && u < pieces) {
-        v[j] = __ldg(reinterpret_cast<const uint4*>(p.qw + (size_t)n * rb) + u);
-        s[j] = __ldg(reinterpret_cast<const unsigned short*>(p.sfr + (size_t)n * sb) + u);
-      } else {
-        v[j] = make_uint4(0u, 0u, 0u, 0u);
-        s[j] = 0u;
-      }
-    }
-  };
-  load_pass(w0, 0, wv[0], ws2[0]);
-  load_pass(w0 + W, 0, wv[1], ws2[1]);
+  RowPrefetch f;
+  prefetch_rows(p, w0, W, lane, f);
 
   griddep_wait();
   if (tid == 0) griddep_launch_dependents();
@@ -207,79 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_nvfp4_kernel(const GvParams 
     if (i < MT * sb) sa[i] = sbv[c] == 0xFFFFFFFFu ? 0.0f : e4m3_to_f(sbv[c]);
   }
   __syncthreads();
-
-  const int passes = (pieces + kPass - 1) / kPass;
-  for (int n0 = w0; n0 < p.N; n0 += 2 * W) {
-    float acc[2][MT];
-#pragma unroll
-    for (int r = 0; r < 2; ++r)
-#pragma unroll
-      for (int m = 0; m < MT; ++m) acc[r][m] = 0.0f;
-    for (int pass = 0; pass < passes; ++pass) {
-      if (n0 != w0 || pass != 0) {
-        load_pass(n0, pass, wv[0], ws2[0]);
-        load_pass(n0 + W, pass, wv[1], ws2[1]);
-      }
-#pragma unroll
-      for (int j = 0; j < kPieces; ++j) {
-        const int u = pass * kPass + j * 32 + lane;
-        if (u >= pieces) break;
-        const int k0 = 32 * u;
-        const uint4* ap = reinterpret_cast<const uint4*>(act + act_slot(k0));
-        float2 sav[MT];
-#pragma unroll
-        for (int m = 0; m < MT; ++m) sav[m] = *reinterpret_cast<const float2*>(sa + m * sb + 2 * u);
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const uint32_t wb[4] = {wv[r][j].x, wv[r][j].y, wv[r][j].z, wv[r][j].w};
-          uint32_t wf[4][4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) e2m1x8_to_f16x8(wb[q], wf[q]);
-          const float2 sw = make_float2(e4m3_to_f(ws2[r][j] & 0xFF), e4m3_to_f(ws2[r][j] >> 8));
-#pragma unroll
-          for (int m = 0; m < MT; ++m) {
-            uint32_t h0 = 0u, h1 = 0u;                       // +0.0 in both halves
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 a = ap[m * (kgrp / 8) + q * 32];
-              const uint32_t av[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-              for (int b = 0; b < 4; ++b) {
-                if (q < 2) h0 = hfma2(wf[q][b], av[b], h0);
-                else h1 = hfma2(wf[q][b], av[b], h1);
-              }
-            }
-            acc[r][m] = fmaf(f16x2_sum(h0), sav[m].x * sw.x, acc[r][m]);
-            acc[r][m] = fmaf(f16x2_sum(h1), sav[m].y * sw.y, acc[r][m]);
-          }
-        }
-      }
-    }
-    // Rank-R term, then the warp reductions (fixed tree) and the store.
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int n = n0 + r * W;
-      if (n >= p.N) break;                                 // warp-uniform
-      float l[MT];
-#pragma unroll
-      for (int m = 0; m < MT; ++m) l[m] = 0.0f;
-      for (int rr = lane; rr < p.R; rr += 32) {
-        const float pv = __bfloat162float(p.pu[(size_t)n * p.R + rr]);
-#pragma unroll
-        for (int m = 0; m < MT; ++m) l[m] = fmaf(lr[m * p.R + rr], pv, l[m]);
-      }
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        float a = acc[r][m], b = l[m];
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-          a += __shfl_xor_sync(0xffffffffu, a, o);
-          b += __shfl_xor_sync(0xffffffffu, b, o);
-        }
-        if (lane == m && m < p.M) p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(fmaf(p.alpha[n], a, b));
-      }
-    }
-  }
+  dot_rows<MT>(p, act, sa, lr, kgrp, w0, W, lane, f);
 }
 
 template <int MT>
@@ -338,3 +374,4 @@ cudaError_t launch_gemv_nvfp4(const GemvLaunch& L, cudaStream_t stream) {
 }
 
 }  // namespace svdq
+

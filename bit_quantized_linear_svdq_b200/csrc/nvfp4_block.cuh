@@ -124,6 +124,53 @@ __device__ __forceinline__ uint32_t quant_block_slow(const uint64_t (&v)[8], uin
   return sb;
 }
 
+// Two-op division for activations: a / b for two lanes from b's reciprocal
+// pair (yh, yl) = (RZ(1/b), RN(1/b - RZ(1/b)) carrying the sign of yh):
+// RN(a*yh + RN(a*yl)), the correctly rounded quotient for every operand pair
+// the activation quantizers meet (bf16 / bf16 smoothing, fp32 / e4m3 codes,
+// fp32 / 6 scales; exhaustive checks in the tests), with zeros carrying the
+// sign of a/b.
+__device__ __forceinline__ uint64_t div_rr2(uint64_t a, uint64_t yh, uint64_t yl) {
+  return fma2(a, yh, mul2(a, yl));
+}
+
+// {RZ(1/b), RN(1/b - RZ(1/b)) with the sign of RZ(1/b)} for a finite nonzero b.
+__device__ __forceinline__ float2 recip_pair(float b) {
+  const double inv = 1.0 / static_cast<double>(b);
+  const float yh = __double2float_rz(inv);
+  const float yl = __double2float_rn(inv - static_cast<double>(yh));
+  return make_float2(yh, copysignf(fabsf(yl), yh));
+}
+
+// One 16-element block of finite values with two-op divisions, the scale's
+// reciprocal pair formed per block (the few-row quantizers): returns the
+// scale byte and the codes (w0: elements 0-7, w1: 8-15).  (yh6, yl6) is
+// recip_pair(6).
+__device__ __forceinline__ uint32_t quant_block_rp(const uint64_t (&v)[8], float amax, float yh6, float yl6,
+                                                   uint32_t& w0, uint32_t& w1) {
+  const float q6 = fmaf(amax, yh6, amax * yl6);       // amax / 6, correctly rounded
+  const uint32_t sb = cvt_e4m3(q6);
+  const float2 sr = sb ? recip_pair(e4m3_to_f32(sb)) : make_float2(0.0f, 0.0f);
+  const uint64_t yh = pk2(sr.x, sr.x), yl = pk2(sr.y, sr.y);
+  uint64_t q[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) q[i] = div_rr2(v[i], yh, yl);
+  const uint32_t keep = sb != 0u ? 0xFFFFFFFFu : 0u;
+  w0 = keep & cvt_e2m1x8(lo2(q[0]), hi2(q[0]), lo2(q[1]), hi2(q[1]), lo2(q[2]), hi2(q[2]), lo2(q[3]), hi2(q[3]));
+  w1 = keep & cvt_e2m1x8(lo2(q[4]), hi2(q[4]), lo2(q[5]), hi2(q[5]), lo2(q[6]), hi2(q[6]), lo2(q[7]), hi2(q[7]));
+  return sb;
+}
+
+// x / smooth for 2N channels (bf16 words xin) with the IEEE divide: the path
+// for blocks whose fast quotients overflowed or hold NaN.
+template <int N>
+__device__ __forceinline__ void smooth_ieee(const uint32_t (&xin)[N], const float* lamf, int k, uint64_t (&v)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+    v[i] = pk2(__fdiv_rn(__uint_as_float(xin[i] << 16), lamf[k + 2 * i]),
+               __fdiv_rn(__uint_as_float(xin[i] & 0xFFFF0000u), lamf[k + 2 * i + 1]));
+}
+
 __device__ __forceinline__ uint32_t quantize_any(const uint64_t (&v)[8], const float2* srec, float y6, uint32_t& w0,
                                                  uint32_t& w1) {
   const float amax = amax8(v);

@@ -111,19 +111,6 @@ struct QTables {
   float2 srec[128];
 };
 
-// a / b for two lanes from b's reciprocal pair (yh, yl): RN(a*yh + RN(a*yl)).
-__device__ __forceinline__ uint64_t div_rr2(uint64_t a, uint64_t yh, uint64_t yl) {
-  return fma2(a, yh, mul2(a, yl));
-}
-
-// {RZ(1/b), RN(1/b - RZ(1/b)) with the sign of RZ(1/b)} for a finite nonzero b.
-__device__ __forceinline__ float2 recip_pair(float b) {
-  const double inv = 1.0 / static_cast<double>(b);
-  const float yh = __double2float_rz(inv);
-  const float yl = __double2float_rn(inv - static_cast<double>(yh));
-  return make_float2(yh, copysignf(fabsf(yl), yh));
-}
-
 // Byte offset, inside one stage's x tile, of the 16-byte group `c` (8 bf16,
 // K elements 8c..8c+7 of the chunk) of row `row`: two 64-column boxes, each
 // 128 rows x 128 bytes with the 128-byte swizzle (16B group index XOR row%8).
@@ -147,16 +134,6 @@ __device__ __forceinline__ uint32_t quant_block_rr(const uint64_t (&v)[8], float
   w0 = keep & cvt_e2m1x8(lo2(q[0]), hi2(q[0]), lo2(q[1]), hi2(q[1]), lo2(q[2]), hi2(q[2]), lo2(q[3]), hi2(q[3]));
   w1 = keep & cvt_e2m1x8(lo2(q[4]), hi2(q[4]), lo2(q[5]), hi2(q[5]), lo2(q[6]), hi2(q[6]), lo2(q[7]), hi2(q[7]));
   return sb;
-}
-
-// x / smooth for 2N channels (bf16 words xin) with the IEEE divide: the path
-// for blocks whose fast quotients overflowed or hold NaN.
-template <int N>
-__device__ __forceinline__ void smooth_ieee(const uint32_t (&xin)[N], const float* lamf, int k, uint64_t (&v)[N]) {
-#pragma unroll
-  for (int i = 0; i < N; ++i)
-    v[i] = pk2(__fdiv_rn(__uint_as_float(xin[i] << 16), lamf[k + 2 * i]),
-               __fdiv_rn(__uint_as_float(xin[i] & 0xFFFF0000u), lamf[k + 2 * i + 1]));
 }
 
 // The IEEE path of one unrotated block (values that overflowed or hold NaN),

@@ -46,49 +46,28 @@ struct FewParams {
   int M, K, Kp, R, ka_pad;
 };
 
-__device__ __forceinline__ uint64_t div_rr2(uint64_t a, uint64_t yh, uint64_t yl) {
-  return fma2(a, yh, mul2(a, yl));
-}
-
-__device__ __forceinline__ float2 recip_pair_f(float b) {
-  const double inv = 1.0 / static_cast<double>(b);
-  const float yh = __double2float_rz(inv);
-  const float yl = __double2float_rn(inv - static_cast<double>(yh));
-  return make_float2(yh, copysignf(fabsf(yl), yh));
-}
-
-// Scale byte and codes of one block of finite values (two-op divisions; the
-// scale's reciprocal pair is formed in double, exactly as the tiled kernel's table).
-__device__ __forceinline__ uint32_t quant16(const uint64_t (&v)[8], float amax, float yh6, float yl6, uint32_t& w0,
-                                            uint32_t& w1) {
-  const float q6 = fmaf(amax, yh6, amax * yl6);
-  const uint32_t sb = cvt_e4m3(q6);
-  const float2 sr = sb ? recip_pair_f(e4m3_to_f32(sb)) : make_float2(0.0f, 0.0f);
-  const uint64_t yh = pk2(sr.x, sr.x), yl = pk2(sr.y, sr.y);
-  uint64_t q[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) q[i] = div_rr2(v[i], yh, yl);
-  const uint32_t keep = sb != 0u ? 0xFFFFFFFFu : 0u;
-  w0 = keep & cvt_e2m1x8(lo2(q[0]), hi2(q[0]), lo2(q[1]), hi2(q[1]), lo2(q[2]), hi2(q[2]), lo2(q[3]), hi2(q[3]));
-  w1 = keep & cvt_e2m1x8(lo2(q[4]), hi2(q[4]), lo2(q[5]), hi2(q[5]), lo2(q[6]), hi2(q[6]), lo2(q[7]), hi2(q[7]));
-  return sb;
-}
-
-// x / smooth for 2N channels with the divide unit.
-template <int N>
-__device__ __forceinline__ void smooth_ieee_n(const uint32_t (&xin)[N], const float* lamf, int k, uint64_t (&v)[N]) {
-#pragma unroll
-  for (int i = 0; i < N; ++i)
-    v[i] = pk2(__fdiv_rn(__uint_as_float(xin[i] << 16), lamf[k + 2 * i]),
-               __fdiv_rn(__uint_as_float(xin[i] & 0xFFFF0000u), lamf[k + 2 * i + 1]));
-}
-
 template <bool ROT>
 __global__ void __launch_bounds__(kFewThreads) quantize_few_kernel(const FewParams p) {
   __shared__ float xs[kGemvMaxRows][kSlice];          // x of the slice, every row
   __shared__ float lsum[kFewThreads / 32][kGemvMaxRows][32];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int k0 = blockIdx.x * kSlice;
+  // The smoothing operands of warp 0's blocks and this thread's first rank
+  // row of P^T are library-owned weights, written at create: requested
+  // before the dependency wait, so only x is read after it.
+  constexpr int kLamPre = ROT ? 16 : 8;
+  float4 lam_pre[kLamPre];
+  if (warp == 0) {
+    const int kl = ROT ? (k0 + 32 * (lane & 3)) / 2 : (k0 + 16 * (lane & 7)) / 2;
+#pragma unroll
+    for (int i = 0; i < kLamPre; ++i) lam_pre[i] = __ldg(p.lamq + lam_slot(kl + i));
+  }
+  uint4 pd_pre[4];
+  if (lane < p.R) {
+    const uint4* prow = reinterpret_cast<const uint4*>(p.pdT + (size_t)lane * p.Kp + k0 + 32 * warp);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) pd_pre[c] = __ldg(prow + c);
+  }
   griddep_wait();                                     // x may be the previous kernel's output
   // x of the slice as fp32 (zeros beyond K and for rows beyond M).
   for (int i = tid; i < kGemvMaxRows * kSlice / 2; i += kFewThreads) {
@@ -103,7 +82,7 @@ __global__ void __launch_bounds__(kFewThreads) quantize_few_kernel(const FewPara
 
   // ---- codes and scales (warp 0)
   if (warp == 0) {
-    const float2 r6 = recip_pair_f(6.0f);
+    const float2 r6 = recip_pair(6.0f);
     if (!ROT) {
       const int m = lane >> 3, j = lane & 7;               // row, 16-channel block
       const int k = k0 + 16 * j;
@@ -117,15 +96,15 @@ __global__ void __launch_bounds__(kFewThreads) quantize_few_kernel(const FewPara
       uint64_t v[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float4 l = p.lamq[lam_slot(k / 2 + i)];
+        const float4 l = lam_pre[i];
         v[i] = div_rr2(bf16x2_to_f2(xin[i]), pk2(l.x, l.y), pk2(l.z, l.w));
       }
       const float amax = amax8(v);
       uint32_t w0, w1, sb;
       if (amax < 3.0e38f) {
-        sb = quant16(v, amax, r6.x, r6.y, w0, w1);
+        sb = quant_block_rp(v, amax, r6.x, r6.y, w0, w1);
       } else {
-        smooth_ieee_n(xin, p.lamf, k, v);
+        smooth_ieee(xin, p.lamf, k, v);
         sb = quant_block_slow(v, w0, w1);
       }
       if (m < p.M) {
@@ -150,11 +129,11 @@ __global__ void __launch_bounds__(kFewThreads) quantize_few_kernel(const FewPara
       float big = 0.0f;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float4 l = p.lamq[lam_slot(kq / 2 + i)];
+        const float4 l = lam_pre[i];
         v[i] = div_rr2(bf16x2_to_f2(xin[i]), pk2(l.x, l.y), pk2(l.z, l.w));
         big = amax_nan(amax_nan(big, lo2(v[i])), hi2(v[i]));
       }
-      if (!(big < 3.0e38f)) smooth_ieee_n(xin, p.lamf, kq, v);
+      if (!(big < 3.0e38f)) smooth_ieee(xin, p.lamf, kq, v);
       hadamard128_quarter(v, qq);
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
@@ -164,7 +143,7 @@ __global__ void __launch_bounds__(kFewThreads) quantize_few_kernel(const FewPara
         const float amax = amax8(blk);
         uint32_t w0, w1, sb;
         if (amax < 3.0e38f)
-          sb = quant16(blk, amax, r6.x, r6.y, w0, w1);
+          sb = quant_block_rp(blk, amax, r6.x, r6.y, w0, w1);
         else
           sb = quant_block_slow(blk, w0, w1);
         const int k = kq + 16 * b;
@@ -193,7 +172,7 @@ __global__ void __launch_bounds__(kFewThreads) quantize_few_kernel(const FewPara
       const uint4* prow = reinterpret_cast<const uint4*>(p.pdT + (size_t)r * p.Kp + k0 + 32 * q);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const uint4 pw = __ldg(prow + c);
+        const uint4 pw = r0 == 0 ? pd_pre[c] : __ldg(prow + c);
         const uint32_t pv[4] = {pw.x, pw.y, pw.z, pw.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {

@@ -366,6 +366,25 @@ def test_zero_alpha_columns(M, kernel, monkeypatch):
     assert_y_close(y[:, zero_cols], lr[:, zero_cols], "zero-alpha columns")
 
 
+@pytest.mark.parametrize("M,K,N,R,rot", [
+    (1, 4096, 512, 32, 0),
+    (2, 384, 300, 16, 0),       # three slices, ragged N
+    (3, 1024, 256, 32, 128),    # rotation
+    (4, 12288, 200, 16, 128),   # three 4096-element passes, rotation
+    (4, 128, 64, 32, 0),        # one slice
+    (1, 2176, 136, 32, 0),      # 17 slices
+])
+def test_few_row_path(M, K, N, R, rot):
+    """1..4 rows (few-row quantizer + CUDA-core matrix-vector product) on
+    shapes that cover 1..17 slices, rotation, K over three 4096-element
+    passes and ragged N: y matches the oracle and repeats bit for bit."""
+    ck = synthetic.make_checkpoint(M, K, N, R, seed=3 * M + K + N, rotate_block=rot, dense_weight=bool(rot),
+                                   wcscales="uniform", wtscale=0.75, name=f"few_{M}x{K}x{N}_r{R}_rot{rot}")
+    layer = make_layer(ck)
+    y1 = check_forward(layer, ck)
+    assert torch.equal(layer.forward(dev_bf16(ck.x)), y1)
+
+
 def test_unfoldable_alpha_takes_plain_epilogue(monkeypatch):
     """wtscale = 2^-30 is outside the range where proj_up / alpha keeps bf16
     precision, so the layer keeps alpha in the epilogue (the 128 x 128 kernel:
