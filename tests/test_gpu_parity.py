@@ -329,6 +329,7 @@ def _select_gemm(kernel, monkeypatch):
     (520, 512, 384, 96, 128),   # pair tiles with two rank boxes, three stages, rotation
     (20, 512, 300, 32, 0),      # 9..32 rows: y^T on 128-column tiles, ragged N
     (29, 768, 136, 16, 128),    # the same with rotation, R = 16
+    (12, 1280, 256, 32, 0),     # y^T tiles, five K steps, two tiles
     (2, 4096, 1000, 32, 0),     # 1..4 rows: CUDA-core product, ragged N
     (4, 9216, 300, 64, 128),    # the same over three 4096-element passes, rotation, R = 64
     (3, 1040, 77, 16, 0),       # K % 32 == 16 (half-masked last piece), R = 16
