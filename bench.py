@@ -64,6 +64,14 @@ def gemm_bytes(M, K, N, R):
     return M * K / 2 + M * K / 16 + 2.0 * M * R + N * K / 2 + N * K / 16 + 2.0 * N * R + 4.0 * N + 2.0 * M * N
 
 
+def gemm_roofline_bound(M, K, N, R, hbm_gbs, fp4_tflops):
+    """The GEMM's roofline bound: "hbm" when its bytes at HBM bandwidth take
+    longer than its flops at the FP4 peak (few rows: the weight read), else
+    "tensor"."""
+    flops = 2.0 * M * N * K + 2.0 * M * N * R
+    return "hbm" if gemm_bytes(M, K, N, R) / (hbm_gbs * 1e9) > flops / (fp4_tflops * 1e12) else "tensor"
+
+
 def source_digest(path):
     """sha256 over a kernel source and every local device header (.cuh) it
     includes, transitively, in first-seen order.  Headers of host-side
@@ -510,7 +518,7 @@ def run_ours(args, world, rank, local):
     g_tf = g_flops / (us_g * 1e-6) / 1e12
     # The GEMM's roofline bound: the slower of its flops at the FP4 peak and
     # its bytes at HBM bandwidth (few rows: the weight read).
-    gemm_bound = "hbm" if gemm_bytes(M, K, N, R) / (pk["hbm_gbs"] * 1e9) > g_flops / (fp4_peak * 1e12) else "tensor"
+    gemm_bound = gemm_roofline_bound(M, K, N, R, pk["hbm_gbs"], fp4_peak)
     kernels = {
         "quantize_act": {"us": us_q, "bound": "hbm", "algorithmic_bytes": quant_bytes(M, K, R),
                          "achieved_gbs": q_gbs, "frac_of_hbm": q_gbs / pk["hbm_gbs"],

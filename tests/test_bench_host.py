@@ -35,3 +35,15 @@ def test_source_digest_follows_device_headers_only(tmp_path):
     (tmp_path / "k.cu").write_text('#include "a.cuh"\n#include "decl.h"\nkernel body, changed\n')
     assert bench.source_digest(str(tmp_path / "k.cu")) != d1
 
+
+
+def test_gemm_roofline_bound_follows_rows():
+    """Few rows read the weights (HBM-bound); the headline shape is a dense
+    contraction (tensor-bound); the crossover sits between M = 256 and 1024
+    at K = N = 4096 with the measured peaks (6553 GB/s, 8120 TFLOP/s)."""
+    hbm, fp4 = 6553.0, 8120.0
+    assert bench.gemm_roofline_bound(1, 4096, 4096, 32, hbm, fp4) == "hbm"
+    assert bench.gemm_roofline_bound(16, 4096, 4096, 32, hbm, fp4) == "hbm"
+    assert bench.gemm_roofline_bound(256, 4096, 4096, 32, hbm, fp4) == "hbm"
+    assert bench.gemm_roofline_bound(1024, 4096, 4096, 32, hbm, fp4) == "tensor"
+    assert bench.gemm_roofline_bound(4096, 3072, 3072, 32, hbm, fp4) == "tensor"
