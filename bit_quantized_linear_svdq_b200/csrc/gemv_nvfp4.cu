@@ -48,8 +48,6 @@ constexpr int kWarps = 16, kThreads = 32 * kWarps;
 // split for at most four rows is one cluster of up to 8 CTAs), so that every
 // CTA of this kernel can start, and request its weights, while it runs.
 constexpr int kReserveSms = 8;
-constexpr int kPieces = 4;                 // 16-byte pieces per lane per row per pass (4096 K elements)
-constexpr int kPass = 32 * kPieces;        // pieces per row per pass
 
 struct GvParams {
   const uint8_t* qw;       // (N, Kp/2) weight codes
@@ -63,6 +61,8 @@ struct GvParams {
   const float* alpha;             // (N)
   __nv_bfloat16* y;               // (M, N)
   int M, N, K, Kp, R;
+  unsigned* err;
+  int rpc;                        // weight rows per CTA (a multiple of 4)
 };
 
 // Shared-memory fp16 slot of element k of a token row: within each group of
@@ -99,146 +99,68 @@ __device__ __forceinline__ float f16x2_sum(uint32_t v) {
   return f.x + f.y;
 }
 
-// One pass of 16-byte weight pieces of row n (and their two block-scale
-// bytes each); zeros past N or the row's end.
-__device__ __forceinline__ void load_pass(const GvParams& p, int n, int pass, int lane, uint4 (&v)[kPieces],
-                                          uint32_t (&s)[kPieces]) {
-  const int pieces = p.Kp / 32, rb = p.Kp / 2, sb = p.Kp / 16;
-#pragma unroll
-  for (int j = 0; j < kPieces; ++j) {
-    const int u = pass * kPass + j * 32 + lane;
-    if (n < p.N && u < pieces) {
-      v[j] = __ldg(reinterpret_cast<const uint4*>(p.qw + (size_t)n * rb) + u);
-      s[j] = __ldg(reinterpret_cast<const unsigned short*>(p.sfr + (size_t)n * sb) + u);
-    } else {
-      v[j] = make_uint4(0u, 0u, 0u, 0u);
-      s[j] = 0u;
-    }
-  }
-}
-
-// A warp's first two weight rows (first pass), their proj_up entries (rank
-// r = lane) and alpha.  All are library-owned weights written at create
-// (which synchronizes), so they are requested before the dependency wait and
-// stream in while the previous kernel is still running.
-struct RowPrefetch {
-  uint4 wv[2][kPieces];
-  uint32_t ws2[2][kPieces];
-  float pu[2], al[2];
+// Shared-memory layout of a CTA (byte offsets): the weight rows' barrier and
+// abort flag, codes [rpc][Kp/2], block scales [rpc][Kp/16], proj_up [rpc][R]
+// bf16, alpha [rpc] f32, token rows [MT][kgrp] fp16, token block scales
+// [MT][Kp/16] f32, L [MT][R] f32.
+struct GvLayout {
+  size_t wq, wsf, wpu, wal, act, sa, lr, total;
 };
-
-__device__ __forceinline__ void prefetch_rows(const GvParams& p, int w0, int W, int lane, RowPrefetch& f) {
-  load_pass(p, w0, 0, lane, f.wv[0], f.ws2[0]);
-  load_pass(p, w0 + W, 0, lane, f.wv[1], f.ws2[1]);
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int n = w0 + r * W;
-    f.pu[r] = 0.0f;
-    f.al[r] = 0.0f;
-    if (n < p.N) {
-      if (lane < p.R) f.pu[r] = __bfloat162float(p.pu[(size_t)n * p.R + lane]);
-      f.al[r] = __ldg(p.alpha + n);
-    }
-  }
-}
-
-// The product for the warp's weight rows w0, w0 + W, ... (two at a time),
-// from the token rows in shared memory: act (fp16, act_slot order, kgrp
-// slots per row), sa (fp32 block scales, Kp/16 per row) and lr (L, R per row).
-template <int MT>
-__device__ __forceinline__ void dot_rows(const GvParams& p, const uint16_t* act, const float* sa, const float* lr,
-                                         int kgrp, int w0, int W, int lane, RowPrefetch& f) {
-  const int pieces = p.Kp / 32, sb = p.Kp / 16;
-  const int passes = (pieces + kPass - 1) / kPass;
-  for (int n0 = w0; n0 < p.N; n0 += 2 * W) {
-    float acc[2][MT];
-#pragma unroll
-    for (int r = 0; r < 2; ++r)
-#pragma unroll
-      for (int m = 0; m < MT; ++m) acc[r][m] = 0.0f;
-    for (int pass = 0; pass < passes; ++pass) {
-      if (n0 != w0 || pass != 0) {
-        load_pass(p, n0, pass, lane, f.wv[0], f.ws2[0]);
-        load_pass(p, n0 + W, pass, lane, f.wv[1], f.ws2[1]);
-      }
-#pragma unroll
-      for (int j = 0; j < kPieces; ++j) {
-        const int u = pass * kPass + j * 32 + lane;
-        if (u >= pieces) break;
-        const int k0 = 32 * u;
-        const uint4* ap = reinterpret_cast<const uint4*>(act + act_slot(k0));
-        float2 sav[MT];
-#pragma unroll
-        for (int m = 0; m < MT; ++m) sav[m] = *reinterpret_cast<const float2*>(sa + m * sb + 2 * u);
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const uint32_t wb[4] = {f.wv[r][j].x, f.wv[r][j].y, f.wv[r][j].z, f.wv[r][j].w};
-          uint32_t wf[4][4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) e2m1x8_to_f16x8(wb[q], wf[q]);
-          const float2 sw = make_float2(e4m3_to_f(f.ws2[r][j] & 0xFF), e4m3_to_f(f.ws2[r][j] >> 8));
-#pragma unroll
-          for (int m = 0; m < MT; ++m) {
-            uint32_t h0 = 0u, h1 = 0u;                       // +0.0 in both halves
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 a = ap[m * (kgrp / 8) + q * 32];
-              const uint32_t av[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-              for (int b = 0; b < 4; ++b) {
-                if (q < 2) h0 = hfma2(wf[q][b], av[b], h0);
-                else h1 = hfma2(wf[q][b], av[b], h1);
-              }
-            }
-            acc[r][m] = fmaf(f16x2_sum(h0), sav[m].x * sw.x, acc[r][m]);
-            acc[r][m] = fmaf(f16x2_sum(h1), sav[m].y * sw.y, acc[r][m]);
-          }
-        }
-      }
-    }
-    // Rank-R term, then the warp reductions (fixed tree) and the store.
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int n = n0 + r * W;
-      if (n >= p.N) break;                                 // warp-uniform
-      const float al = n0 == w0 ? f.al[r] : p.alpha[n];
-      float l[MT];
-#pragma unroll
-      for (int m = 0; m < MT; ++m) l[m] = 0.0f;
-      for (int rr = lane; rr < p.R; rr += 32) {
-        const float pv = (n0 == w0 && rr == lane) ? f.pu[r] : __bfloat162float(p.pu[(size_t)n * p.R + rr]);
-#pragma unroll
-        for (int m = 0; m < MT; ++m) l[m] = fmaf(lr[m * p.R + rr], pv, l[m]);
-      }
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        float a = acc[r][m], b = l[m];
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-          a += __shfl_xor_sync(0xffffffffu, a, o);
-          b += __shfl_xor_sync(0xffffffffu, b, o);
-        }
-        if (lane == m && m < p.M) p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(fmaf(al, a, b));
-      }
-    }
-  }
+__host__ __device__ inline GvLayout gv_layout(int MT, int Kp, int R, int rpc) {
+  GvLayout l;
+  const size_t kgrp = (size_t)(Kp + 1023) / 1024 * 1024;
+  l.wq = 16;
+  l.wsf = l.wq + (size_t)rpc * (Kp / 2);
+  l.wpu = l.wsf + (size_t)rpc * (Kp / 16);
+  l.wal = l.wpu + (size_t)rpc * R * 2;
+  l.act = l.wal + (size_t)rpc * 4;
+  l.sa = l.act + (size_t)MT * kgrp * 2;
+  l.lr = l.sa + (size_t)MT * (Kp / 16) * 4;
+  l.total = l.lr + (size_t)MT * R * 4;
+  return l;
 }
 
 template <int MT>
 __global__ void __launch_bounds__(kThreads, 1) gemv_nvfp4_kernel(const GvParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
+  const GvLayout Ls = gv_layout(MT, p.Kp, p.R, p.rpc);
   const int kgrp = (p.Kp + 1023) & ~1023;                  // fp16 slots per token row
-  uint16_t* act = reinterpret_cast<uint16_t*>(smem);        // [MT][kgrp] fp16
-  float* sa = reinterpret_cast<float*>(act + MT * kgrp);    // [MT][Kp/16] block scales (0 beyond K)
-  float* lr = sa + MT * (p.Kp / 16);                        // [MT][R]
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int W = gridDim.x * kWarps, w0 = blockIdx.x * kWarps + warp;
   const int rb = p.Kp / 2, sb = p.Kp / 16;                  // row bytes: codes, scales
   const int K16 = p.K / 16;
+  uint64_t* wbar = reinterpret_cast<uint64_t*>(smem);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 8);
+  const uint8_t* wq = smem + Ls.wq;
+  const uint8_t* wsf = smem + Ls.wsf;
+  const __nv_bfloat16* wpu = reinterpret_cast<const __nv_bfloat16*>(smem + Ls.wpu);
+  const float* wal = reinterpret_cast<const float*>(smem + Ls.wal);
+  uint16_t* act = reinterpret_cast<uint16_t*>(smem + Ls.act);   // [MT][kgrp] fp16
+  float* sa = reinterpret_cast<float*>(smem + Ls.sa);            // [MT][Kp/16] block scales (0 beyond K)
+  float* lr = reinterpret_cast<float*>(smem + Ls.lr);            // [MT][R]
 
-  RowPrefetch f;
-  prefetch_rows(p, w0, W, lane, f);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_begin = blockIdx.x * p.rpc;
+  const int rows = max(0, min(p.rpc, p.N - n_begin));
+
+  // This CTA's weight rows -> shared memory by bulk copies: library-owned
+  // weights written at create, so requested before the dependency wait; the
+  // copy engine streams them while the previous kernel runs and leaves the
+  // load path free for the token rows after the wait.  Scale rows are copied
+  // in pairs and alpha in fours (their buffers are padded so).
+  if (tid == 0) {
+    mbar_init(smem_u32(wbar), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    if (rows > 0) {
+      const int rows2 = (rows + 1) & ~1, rows4 = (rows + 3) & ~3;
+      const uint32_t wb = smem_u32(wbar);
+      mbar_arrive_expect_tx(wb, (uint32_t)((size_t)rows * rb + (size_t)rows2 * sb + (size_t)rows * p.R * 2 +
+                                           (size_t)rows4 * 4));
+      bulk_load(smem_u32(wq), p.qw + (size_t)n_begin * rb, (uint32_t)((size_t)rows * rb), wb);
+      bulk_load(smem_u32(wsf), p.sfr + (size_t)n_begin * sb, (uint32_t)((size_t)rows2 * sb), wb);
+      bulk_load(smem_u32(wpu), p.pu + (size_t)n_begin * p.R, (uint32_t)((size_t)rows * p.R * 2), wb);
+      bulk_load(smem_u32(wal), p.alpha + n_begin, (uint32_t)(rows4 * 4), wb);
+    }
+  }
 
   griddep_wait();
   if (tid == 0) griddep_launch_dependents();
@@ -314,8 +236,83 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_nvfp4_kernel(const GvParams 
     const int i = tid + c * kThreads;
     if (i < MT * sb) sa[i] = sbv[c] == 0xFFFFFFFFu ? 0.0f : e4m3_to_f(sbv[c]);
   }
-  __syncthreads();
-  dot_rows<MT>(p, act, sa, lr, kgrp, w0, W, lane, f);
+  __syncthreads();                                          // token rows staged; barrier initialized
+  // The weight rows have landed (bounded wait; on expiry the CTA records an
+  // error and stores nothing).
+  const bool have = rows == 0 || wait_bounded(smem_u32(wbar), 0, abort_flag, p.err, kErrGemmTimeout);
+  if (!__syncthreads_and(have)) return;
+
+  // The product: warp w takes local rows w, w + 16, ... two at a time; lane
+  // l reads 16-byte pieces l, l + 32, ... of a row.
+  const int pieces = p.Kp / 32;
+  for (int i0 = warp; i0 < rows; i0 += 2 * kWarps) {
+    const bool two = i0 + kWarps < rows;
+    float acc[2][MT];
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) acc[r][m] = 0.0f;
+    for (int u = lane; u < pieces; u += 32) {
+      const int k0 = 32 * u;
+      const uint4* ap = reinterpret_cast<const uint4*>(act + act_slot(k0));
+      float2 sav[MT];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) sav[m] = *reinterpret_cast<const float2*>(sa + m * sb + 2 * u);
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        if (r == 1 && !two) break;
+        const int i = i0 + r * kWarps;
+        const uint4 wv = *reinterpret_cast<const uint4*>(wq + (size_t)i * rb + 16 * u);
+        const uint32_t ws2 = *reinterpret_cast<const unsigned short*>(wsf + (size_t)i * sb + 2 * u);
+        const uint32_t wb[4] = {wv.x, wv.y, wv.z, wv.w};
+        uint32_t wf[4][4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) e2m1x8_to_f16x8(wb[q], wf[q]);
+        const float2 sw = make_float2(e4m3_to_f(ws2 & 0xFF), e4m3_to_f(ws2 >> 8));
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          uint32_t h0 = 0u, h1 = 0u;                       // +0.0 in both halves
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 a = ap[m * (kgrp / 8) + q * 32];
+            const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int b2 = 0; b2 < 4; ++b2) {
+              if (q < 2) h0 = hfma2(wf[q][b2], av[b2], h0);
+              else h1 = hfma2(wf[q][b2], av[b2], h1);
+            }
+          }
+          acc[r][m] = fmaf(f16x2_sum(h0), sav[m].x * sw.x, acc[r][m]);
+          acc[r][m] = fmaf(f16x2_sum(h1), sav[m].y * sw.y, acc[r][m]);
+        }
+      }
+    }
+    // Rank-R term, then the warp reductions (fixed tree) and the store.
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      if (r == 1 && !two) break;                            // warp-uniform
+      const int i = i0 + r * kWarps;
+      float l[MT];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) l[m] = 0.0f;
+      for (int rr = lane; rr < p.R; rr += 32) {
+        const float pv = __bfloat162float(wpu[(size_t)i * p.R + rr]);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) l[m] = fmaf(lr[m * p.R + rr], pv, l[m]);
+      }
+      const float al = wal[i];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        float a = acc[r][m], b = l[m];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+          a += __shfl_xor_sync(0xffffffffu, a, o);
+          b += __shfl_xor_sync(0xffffffffu, b, o);
+        }
+        if (lane == m && m < p.M) p.y[(size_t)m * p.N + n_begin + i] = __float2bfloat16_rn(fmaf(al, a, b));
+      }
+    }
+  }
 }
 
 template <int MT>
@@ -337,10 +334,25 @@ cudaError_t launch_mt(const GvParams& p, int grid, size_t smem, cudaStream_t str
 
 }  // namespace
 
+namespace {
+
+// Weight rows per CTA: enough that the grid (all but kReserveSms SMs) covers
+// N, a multiple of 4, and no more than shared memory allows.
+int gemv_rpc(int M, int N, int Kp, int R, int num_sms) {
+  const int mt = M <= 1 ? 1 : (M <= 2 ? 2 : 4);
+  const int ctas = std::max(1, num_sms - kReserveSms);
+  int rpc = ((N + ctas - 1) / ctas + 3) & ~3;
+  while (rpc > 4 && gv_layout(mt, Kp, R, rpc).total > 200 * 1024) rpc -= 4;
+  return rpc;
+}
+
+}  // namespace
+
+// Shared memory with the fewest weight rows per CTA (4): the product applies
+// when that fits.
 size_t gemv_smem_bytes(int M, int Kp, int R) {
   const int mt = M <= 1 ? 1 : (M <= 2 ? 2 : 4);
-  const size_t kgrp = (size_t)(Kp + 1023) / 1024 * 1024;
-  return (size_t)mt * (kgrp * 2 + (size_t)(Kp / 16) * 4 + (size_t)R * 4);
+  return gv_layout(mt, Kp, R, 4).total;
 }
 
 bool gemv_applies(int M, int Kp, int R) {
@@ -366,8 +378,11 @@ cudaError_t launch_gemv_nvfp4(const GemvLaunch& L, cudaStream_t stream) {
   p.K = L.K;
   p.Kp = L.Kp;
   p.R = L.R;
-  const int grid = std::max(1, std::min(L.num_sms - kReserveSms, (L.N + kWarps - 1) / kWarps));
-  const size_t smem = gemv_smem_bytes(L.M, L.Kp, L.R);
+  p.err = L.err;
+  p.rpc = gemv_rpc(L.M, L.N, L.Kp, L.R, L.num_sms);
+  const int grid = (L.N + p.rpc - 1) / p.rpc;
+  const int mt = L.M <= 1 ? 1 : (L.M <= 2 ? 2 : 4);
+  const size_t smem = gv_layout(mt, L.Kp, L.R, p.rpc).total;
   if (L.M == 1) return launch_mt<1>(p, grid, smem, stream);
   if (L.M == 2) return launch_mt<2>(p, grid, smem, stream);
   return launch_mt<4>(p, grid, smem, stream);

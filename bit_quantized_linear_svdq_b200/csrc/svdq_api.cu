@@ -370,7 +370,9 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
 
   CREATE_CUDA(cudaMalloc(&h->qw, (size_t)d->N * (h->Kp / 2)));
   CREATE_CUDA(cudaMalloc(&h->sfb, (size_t)n_tiles_even * h->ka_pad * svdq::kSfAtomBytes));
-  CREATE_CUDA(cudaMalloc(&h->sfr, (size_t)d->N * (h->Kp / 16)));
+  // Row-major scales, padded to an even number of rows (the matrix-vector
+  // product copies scale rows in pairs).
+  CREATE_CUDA(cudaMalloc(&h->sfr, (size_t)((d->N + 1) & ~1) * (h->Kp / 16)));
   CREATE_CUDA(cudaMalloc(&h->pdT, (size_t)d->R * h->Kp * 2));
   CREATE_CUDA(cudaMalloc(&h->pu, (size_t)d->N * d->R * 2));
   CREATE_CUDA(cudaMalloc(&h->lamq, (size_t)(h->Kp / 2) * sizeof(float4)));
@@ -393,7 +395,7 @@ svdq_status svdq_linear_create(svdq_linear** out, const svdq_linear_desc* d, voi
   CREATE_CUDA(cudaMemcpy2DAsync(h->qw, h->Kp / 2, d->qweight, d->K / 2, d->K / 2, d->N, cudaMemcpyDeviceToDevice,
                                 stream));
   CREATE_CUDA(cudaMemsetAsync(h->sfb, 0, (size_t)n_tiles_even * h->ka_pad * svdq::kSfAtomBytes, stream));
-  CREATE_CUDA(cudaMemsetAsync(h->sfr, 0, (size_t)d->N * (h->Kp / 16), stream));
+  CREATE_CUDA(cudaMemsetAsync(h->sfr, 0, (size_t)((d->N + 1) & ~1) * (h->Kp / 16), stream));
   prepare_alpha<<<grid_for(Npad), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(d->wcscales),
                                                      static_cast<const __nv_bfloat16*>(d->wtscale), h->alpha, d->N,
                                                      Npad);
@@ -638,6 +640,7 @@ svdq_status forward_gemm(const svdq_linear* h, int M, void* y, void* workspace, 
     v.Kp = h->Kp;
     v.R = h->R;
     v.num_sms = num_sms();
+    v.err = h->err;
     cudaError_t e = svdq::launch_gemv_nvfp4(v, stream);
     if (e != cudaSuccess) return cuda_fail(e, "gemv launch");
     return SVDQ_OK;

@@ -146,6 +146,7 @@ struct GemvLaunch {
   void* y;
   int M, N, K, Kp, R;
   int num_sms;
+  unsigned* err;            // device error word (a bounded wait that expires sets kErrGemmTimeout)
 };
 size_t gemv_smem_bytes(int M, int Kp, int R);
 bool gemv_applies(int M, int Kp, int R);
