@@ -8,15 +8,15 @@
 // most eight multiply-adds, so the time is the weight read from HBM and the
 // kernel is a coalesced stream, not a tensor-core tile loop.
 //
-// Decomposition.  One CTA of 16 warps per SM, on all but 8 SMs (left to the
-// quantizer that runs before it); warp w of the grid owns weight
-// rows w, w + W, w + 2W, ... (W = warps in the grid), two at a time.  Lane l
-// reads 16-byte pieces l, l + 32, ... of a row (32 FP4 codes = two scale
-// blocks each), so every load instruction of a warp covers 512 contiguous
-// bytes.  The token rows are decoded once per CTA into shared memory as fp16
-// (exact: every E2M1 value is an fp16 value), in an order that makes each
-// lane's four 16-byte reads per piece conflict-free; their block scales go to
-// shared memory as fp32.
+// Decomposition.  One CTA of 16 warps owns a contiguous block of rpc weight
+// rows (a multiple of 4), on at most all but 8 SMs (left to the quantizer
+// that runs before it).  Its codes, block scales, proj_up rows and alpha come
+// into shared memory by four bulk copies; warp w takes local rows w, w + 16,
+// ... two at a time, and lane l reads 16-byte pieces l, l + 32, ... of a row
+// (32 FP4 codes = two scale blocks each).  The token rows are decoded once per
+// CTA into shared memory as fp16 (exact: every E2M1 value is an fp16 value),
+// in an order that makes each lane's four 16-byte reads per piece
+// conflict-free; their block scales go to shared memory as fp32.
 //
 // Arithmetic.  cvt.rn.f16x2.e2m1x2 turns a weight byte into two exact fp16
 // values; the 16 products of a scale block go into two fp16 lanes of eight
@@ -29,9 +29,10 @@
 // not depend on timing) and stores y = bf16(fma(alpha, acc, lr)).
 //
 // The weights are library-owned and written once at create time (which
-// synchronizes), so each warp's first two rows are requested before the
-// programmatic-dependent-launch wait and stream in while the previous kernel
-// (the activation quantizer) is still running.
+// synchronizes), so the bulk copies are issued before the
+// programmatic-dependent-launch wait: the copy engine streams them while the
+// previous kernel (the activation quantizer) is still running, the threads
+// reach the wait at once, and after it only the token rows are loaded.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
