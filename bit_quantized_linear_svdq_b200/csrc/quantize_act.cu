@@ -118,6 +118,11 @@ __device__ __forceinline__ uint32_t xoff(int row, int c) {
   return (uint32_t)((c >> 3) * kXBoxBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4));
 }
 
+// XOR mask on the 16-byte group index of a row of the partial-L receive
+// buffer (R fp32 values, R a multiple of 16): 8 groups of a 128-byte row, or
+// the 4 groups of a 64-byte row when R = 16.
+__device__ __forceinline__ int recv_swizzle(int R) { return R >= 32 ? 7 : 3; }
+
 // One 16-element block of finite values -> scale byte + 16 codes (w0: 0-7, w1: 8-15).
 __device__ __forceinline__ uint32_t quant_block_rr(const uint64_t (&v)[8], float amax, const float2* srec, float yh6,
                                                    float yl6, uint32_t& w0, uint32_t& w1) {
@@ -369,7 +374,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_load(smem_u32(LAM + s * kLamStageBytes), p.lamq + kc / 2, kLamStageBytes, fb);
         issued = i + 1;
       };
-      for (int i = 0; i < nch && i < p.stages; ++i) load(i);
+      // The first two chunks go out at once; the rest of the ring only once
+      // chunk 0 has landed.  Every CTA asks for its first chunks at the same
+      // moment, and requests for later stages queued beside them delay some
+      // CTAs' first chunk (their cluster then waits for them at the end).
+      const int first = min(nch, 2);
+      for (int i = 0; i < first; ++i) load(i);
+      if (nch > first && p.stages > first &&
+          wait_bounded(smem_u32(&full[0]), 0, abort_flag, p.err, kErrQuantTimeout))
+        for (int i = first; i < nch && i < p.stages; ++i) load(i);
       for (int j = 0; j < nch; ++j) {
         const int s = j % p.stages, par = (j / p.stages) & 1;
         // Chunk j's codes and scales are staged: write them.
@@ -505,6 +518,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                                                   row % rows_per) * R * 4),
                                                      owner)
                                        : 0u;
+    // The receive buffer's 16-byte groups are XOR-swizzled by buffer row, so
+    // the 32 lanes' stores of one column (32 rows) spread over every bank.
+    const uint32_t gsw = (uint32_t)(((int)cluster_ctarank() * rows_per + row % rows_per) & recv_swizzle(R));
     if (ok) {
       for (int j = 0; j < R; j += 16) {
         uint32_t r[16];
@@ -525,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
           for (int t = 0; t < 4; ++t)
-            st_shared_cluster_v4(dst0 + (uint32_t)(j + 4 * t) * 4u, __uint_as_float(r[4 * t]),
+            st_shared_cluster_v4(dst0 + ((((uint32_t)(j + 4 * t) >> 2) ^ gsw) << 4), __uint_as_float(r[4 * t]),
                                  __uint_as_float(r[4 * t + 1]), __uint_as_float(r[4 * t + 2]),
                                  __uint_as_float(r[4 * t + 3]));
         }
@@ -543,7 +559,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (m >= p.M) continue;
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
         for (int q = 0; q < p.ksplit; ++q) {
-          const float4 v = *reinterpret_cast<const float4*>(recv + (size_t)(q * rows_per + rl) * R + col);
+          const int b = q * rows_per + rl;
+          const float4 v = *reinterpret_cast<const float4*>(recv + (size_t)b * R + 4 * ((col >> 2) ^ (b & recv_swizzle(R))));
           a0 += v.x;
           a1 += v.y;
           a2 += v.z;
