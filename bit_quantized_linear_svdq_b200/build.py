@@ -48,7 +48,9 @@ def _digest(deps) -> str:
     h.update(" ".join(NVCC_FLAGS).encode())
     for d in deps:
         with open(d, "rb") as f:
-            h.update(d.encode())
+            # Paths relative to the repository: a copy of the tree elsewhere
+            # (with its built library) keeps the same digest.
+            h.update(os.path.relpath(d, ROOT).encode())
             h.update(f.read())
     return h.hexdigest()
 

@@ -119,9 +119,11 @@ __device__ __forceinline__ uint32_t xoff(int row, int c) {
 }
 
 // XOR mask on the 16-byte group index of a row of the partial-L receive
-// buffer (R fp32 values, R a multiple of 16): 8 groups of a 128-byte row, or
-// the 4 groups of a 64-byte row when R = 16.
-__device__ __forceinline__ int recv_swizzle(int R) { return R >= 32 ? 7 : 3; }
+// buffer (R fp32 values, R a multiple of 16, so R/4 groups per row): 7 when
+// the groups come in whole blocks of 8 (R a multiple of 32), else 3 (blocks
+// of 4).  The swizzled index stays inside its aligned block, hence inside the
+// row.
+__device__ __forceinline__ int recv_swizzle(int R) { return (R / 4) % 8 == 0 ? 7 : 3; }
 
 // One 16-element block of finite values -> scale byte + 16 codes (w0: 0-7, w1: 8-15).
 __device__ __forceinline__ uint32_t quant_block_rr(const uint64_t (&v)[8], float amax, const float2* srec, float yh6,

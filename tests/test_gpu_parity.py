@@ -326,6 +326,7 @@ def _select_gemm(kernel, monkeypatch):
     (2048, 256, 2560, 32, 0),   # more 256 x 256 tiles than CTA pairs: two tiles per pair
     (260, 512, 300, 32, 0),     # pair tiles with N % 8 != 0: element stores instead of TMA
     (300, 768, 520, 48, 0),     # pair tiles, rank box only partly filled (R = 48 of 64)
+    (40, 640, 200, 112, 0),     # R = 112: 28 groups per partial-L receive row (swizzle mask 3)
     (520, 512, 384, 96, 128),   # pair tiles with two rank boxes, three stages, rotation
     (20, 512, 300, 32, 0),      # 9..32 rows: y^T on 128-column tiles, ragged N
     (29, 768, 136, 16, 128),    # the same with rotation, R = 16
