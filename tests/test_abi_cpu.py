@@ -147,3 +147,24 @@ def test_fp4_loop_rejects_bad_iters_on_host(lib):
     ctas = ctypes.c_int(-1)
     assert lib.svdq_fp4_mma_loop(0, ctypes.byref(ctas), None) == 1
     assert lib.svdq_fp4_mma_loop((1 << 20) + 1, ctypes.byref(ctas), None) == 1
+
+
+def test_build_stamp_is_independent_of_the_tree_location(tmp_path):
+    # The stamp beside the library is a digest of the sources and flags; a copy
+    # of the tree at another path (with its built library) must not rebuild,
+    # and a changed source must.
+    import importlib.util
+    import shutil
+
+    root = tmp_path / "copy"
+    shutil.copytree(B.PKG, root / "bit_quantized_linear_svdq_b200",
+                    ignore=shutil.ignore_patterns("_lib", "__pycache__"))
+    shutil.copytree(f"{B.ROOT}/include", root / "include")
+    spec = importlib.util.spec_from_file_location("build_copy", root / "bit_quantized_linear_svdq_b200" / "build.py")
+    Bc = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(Bc)
+    assert Bc.ROOT == str(root)
+    assert Bc._digest(Bc._sources()[1]) == B._digest(B._sources()[1])
+    with open(root / "bit_quantized_linear_svdq_b200" / "csrc" / "kcommon.cuh", "a") as f:
+        f.write("\n")
+    assert Bc._digest(Bc._sources()[1]) != B._digest(B._sources()[1])
